@@ -1,0 +1,165 @@
+/*
+ * moe.h -- C ABI of the routed sparse-MoE block on B200 (sm_100a).
+ *
+ * What the block computes.  The Strata pages describe one layer of
+ * Qwen3.8-Flash-Next as: a router scores the token against 512 experts and
+ * picks 10, an always-on shared expert runs beside them, and the GPU adds the
+ * results up before the next layer starts ("Strata open-source runtime: a 12GB
+ * card runs the 125B Qwen3 model", section "the model itself"; "Why Strata is
+ * fast on low-VRAM GPUs", sections "the problem" and "one token, three
+ * workers").  Decode checks a verify window of up to 4 tokens in one pass
+ * (same page, "guess first, then check"); prefill reads prompts in chunks of up
+ * to 8192 tokens ("reading long prompts").  Experts are stored as low-bit
+ * group-quantised weights ("the cost": Q2_0 / IQ3 expert files).
+ *
+ * Per token x (bf16, d values):
+ *   logits[e] = sum_i x[i] * Wr[e][i] + b[e]                       (fp32)
+ *   ids       = the top_k largest logits, largest first, equal logits ->
+ *               lower expert index, NaN below every number
+ *   w[j]      = exp(logits[ids[j]] - logits[ids[0]]) / sum over the selected
+ *   FFN_e(x)  = Wd_e (silu(Wg_e x) * (Wu_e x)),  silu(z) = z / (1 + e^-z)
+ *   y         = FFN_shared(x) + sum_j w[j] * FFN_{ids[j]}(x)   -> bf16
+ * with MOE_F_PRENORM the FFNs and the router see bf16(RMSNorm(x)) (eps 1e-6, no
+ * weight) instead of x, and with MOE_F_RESIDUAL the output is x + y.
+ *
+ * Packed expert weights.  Each expert is Wg (ffn x d), Wu (ffn x d), Wd
+ * (d x ffn), each R x K with K contracted, quantised in groups of 32
+ * consecutive K elements: weight = fp16 scale * (code - 2^(bits-1)).
+ *  - rows in tiles of 16; inside a tile, group words ordered group-major:
+ *    word (c, r) at byte (c*16 + r) * 8 of the tile;
+ *  - code j = 8m + 2t + h of a group: low two bits at bit 32h + 8t + 2m of
+ *    the group's 8-byte little-endian word;
+ *  - bits = 3: the high bit of code j at bit 16h + 4t + m of a 4-byte word;
+ *    a tile holds all its 8-byte words (K/32*16*8 bytes), then all its 4-byte
+ *    words in the same (c, r) order;
+ *  - scales: fp16, one per (row, group), element c*16 + r of the tile's
+ *    16*K/32 scales;
+ *  - an expert = Wg tiles, Wu tiles, Wd tiles (codes), and the same order for
+ *    its scales; expert e lives in slot expert_slot[e].
+ *  Bytes per expert: codes 3*ffn*d/32 * (8 | 12), scales 3*ffn*d/32 * 2.
+ *
+ * Conventions for every call below.
+ *  - Pointers marked "dev" are device memory owned by the caller; the library
+ *    never allocates, frees or synchronises.  It enqueues kernels on `stream`
+ *    (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *  - Row-major layouts, token dimension outermost.
+ *  - Validation (null pointers, shapes, alignment, workspace size) happens on
+ *    the host before any launch; a failed check returns its status and
+ *    enqueues nothing.  MOE_OK means "enqueued": asynchronous faults surface
+ *    at the caller's next synchronisation, and the kernels' own checks (bounded
+ *    waits; range checks under MOE_F_DEBUG) set an error word in the
+ *    workspace, read back with moe_workspace_error().
+ *  - The workspace is caller-owned device memory of at least
+ *    moe_workspace_bytes() bytes, 256-byte aligned, zeroed once with
+ *    moe_workspace_init() before first use.  Kernels leave it ready for the
+ *    next call.  Calls sharing one workspace must be ordered (same stream or
+ *    explicit events).
+ *  - Thread-safe for calls on distinct workspaces; stateless otherwise.
+ *  - Limits: d_model % 32 == 0 and 32 <= d_model <= 4096; ffn, shared_ffn %
+ *    32 == 0 and <= 4096; 1 <= top_k <= 16; top_k <= n_experts <= 1024;
+ *    bits in {2, 3}; group == 32.
+ *  - Alignment: x, y, codes, scales, shared_codes, shared_scales, router_w:
+ *    16 bytes.
+ */
+#ifndef MOE_H
+#define MOE_H
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad flag */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* a limit above is not met */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3,
+  MOE_ERR_MISALIGNED = 4,
+  MOE_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
+  MOE_ERR_DEVICE_CHECK = 6,       /* a kernel range check tripped (MOE_F_DEBUG) */
+  MOE_ERR_TIMEOUT = 7,            /* a kernel's bounded wait ran out */
+  MOE_ERR_NO_DEVICE = 8           /* no sm_100 device current */
+} moe_status;
+
+/* flags */
+#define MOE_F_PRENORM 1u        /* router and experts see bf16(RMSNorm(x)) */
+#define MOE_F_RESIDUAL 2u       /* y = x + MoE(.) */
+#define MOE_F_DETERMINISTIC 4u  /* prefill: fixed-order combine (no float atomics) */
+#define MOE_F_DEBUG 8u          /* kernels range-check ids, slots and values */
+
+/* One layer.  A host struct, read only during the call. */
+typedef struct {
+  int32_t d_model;       /* d */
+  int32_t n_experts;     /* E */
+  int32_t ffn;           /* F, routed experts' hidden size */
+  int32_t top_k;         /* k */
+  int32_t bits;          /* 2 or 3 */
+  int32_t group;         /* must be 32 */
+  int32_t shared_ffn;    /* Fs; 0 = no shared expert */
+  const float* router_w;        /* dev fp32 [E][d] */
+  const float* router_bias;     /* dev fp32 [E] or NULL */
+  const int32_t* expert_slot;   /* dev int32 [E]: expert -> slot, a permutation of 0..E-1 */
+  const uint8_t* codes;         /* dev [E slots][3*F*d/32*(8|12)] */
+  const uint16_t* scales;       /* dev fp16 bits [E slots][3*F*d/32] */
+  const uint8_t* shared_codes;  /* dev [3*Fs*d/32*(8|12)] or NULL when Fs == 0 */
+  const uint16_t* shared_scales;/* dev fp16 bits [3*Fs*d/32] or NULL when Fs == 0 */
+} moe_layer;
+
+/* Bytes of workspace the calls below need for up to max_tokens tokens
+ * (0 on invalid arguments). */
+size_t moe_workspace_bytes(const moe_layer* layer, int32_t max_tokens);
+
+/* Zero a workspace (enqueued on stream).  Needed once after allocation. */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Copy the workspace's device error word to *code_out (0 = none) and clear it.
+ * Synchronises `stream` (a debugging aid, not for the hot path).  Returns
+ * MOE_ERR_TIMEOUT / MOE_ERR_DEVICE_CHECK when the word was set. */
+moe_status moe_workspace_error(void* ws, size_t ws_bytes, uint32_t* code_out, void* stream);
+
+/* Router + top-k + softmax renormalisation for T tokens.
+ *  x_bf16: dev bf16 [T][d].  flags: MOE_F_PRENORM and MOE_F_DEBUG honoured.
+ *  logits_or_null: dev fp32 [T][E], written when non-NULL.
+ *  topk_ids: dev int32 [T][k] (largest first); topk_w: dev fp32 [T][k].
+ *  T = 0 enqueues nothing. */
+moe_status moe_route_topk(const moe_layer* layer, const void* x_bf16, int32_t T, uint32_t flags,
+                          float* logits_or_null, int32_t* topk_ids, float* topk_w, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/* Decode / verify-window expert step for 1 <= T <= 8 tokens: the selected
+ * experts (deduplicated across the window) and the shared expert, combined
+ * with the routing weights.  Weight bytes are streamed once per call.
+ *  topk_ids/topk_w: dev, as written by moe_route_topk.  y_bf16: dev bf16 [T][d]
+ *  (may not alias x).  flags: PRENORM, RESIDUAL, DEBUG. */
+moe_status moe_expert_ffn_decode(const moe_layer* layer, const void* x_bf16, int32_t T,
+                                 const int32_t* topk_ids, const float* topk_w, void* y_bf16,
+                                 uint32_t flags, void* ws, size_t ws_bytes, void* stream);
+
+/* Prefill expert step for T >= 1 tokens: tokens bucketed per expert (ascending
+ * token order inside each expert), tensor-core grouped GEMMs with the
+ * dequantisation fused into the operand tiles, shared expert over all tokens,
+ * routing-weighted combine.
+ *  bucket_offsets_or_null: dev int32 [E+1], written when non-NULL (exclusive
+ *  scan of per-expert counts).  bucket_entries_or_null: dev int32 [T*k],
+ *  written when non-NULL: for each expert its entries t*k + j, tokens
+ *  ascending.  flags: PRENORM, RESIDUAL, DETERMINISTIC, DEBUG. */
+moe_status moe_expert_ffn_prefill(const moe_layer* layer, const void* x_bf16, int32_t T,
+                                  const int32_t* topk_ids, const float* topk_w, void* y_bf16,
+                                  int32_t* bucket_offsets_or_null, int32_t* bucket_entries_or_null,
+                                  uint32_t flags, void* ws, size_t ws_bytes, void* stream);
+
+/* The whole block: moe_route_topk, then the decode step for T <= 4 and the
+ * prefill step otherwise.  Routing lists live in the workspace. */
+moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t T, void* y_bf16,
+                             uint32_t flags, void* ws, size_t ws_bytes, void* stream);
+
+const char* moe_status_string(moe_status status);
+
+/* Library build information (a static string). */
+const char* moe_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

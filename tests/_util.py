@@ -1,0 +1,109 @@
+"""Helpers shared by the GPU parity tests."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from routed_expert_ffn_06_b200 import moe, synth
+
+# Tolerances of the block output against the fp64 oracle.
+MAX_REL = 2e-2   # per token: max_i |y - ŷ| / max_i |ŷ|, worst token
+RMS_REL = 3e-3   # ||y - ŷ||_2 / ||ŷ||_2 over the whole output
+
+
+def errors(y_gpu, y_ref):
+    """(max rel, rms rel) of a device output against the oracle's fp64."""
+    y = y_gpu.float().cpu().double().numpy() if torch.is_tensor(y_gpu) else np.asarray(y_gpu)
+    r = np.asarray(y_ref, dtype=np.float64)
+    diff = y - r
+    per_tok = np.abs(diff).max(axis=1) / np.maximum(np.abs(r).max(axis=1), 1e-30)
+    rms = np.linalg.norm(diff) / max(np.linalg.norm(r), 1e-30)
+    return float(per_tok.max()), float(rms)
+
+
+def assert_close(y_gpu, y_ref, max_rel=MAX_REL, rms_rel=RMS_REL):
+    mr, rr = errors(y_gpu, y_ref)
+    assert mr <= max_rel and rr <= rms_rel, f"max rel {mr:.3e} (<= {max_rel}), rms rel {rr:.3e} (<= {rms_rel})"
+    return mr, rr
+
+
+def logit_bound(layer, x_in: np.ndarray) -> np.ndarray:
+    """1e-4 * (sum_i |x_i Wr_ei| + |b_e|): the fp32 logit tolerance."""
+    Wr = np.abs(layer.router_w.double().cpu().numpy())
+    b = 0.0 if layer.router_bias is None else np.abs(layer.router_bias.double().cpu().numpy())
+    return 1e-4 * (np.abs(x_in) @ Wr.T + b)
+
+
+def bf16_bits(x: torch.Tensor) -> np.ndarray:
+    return x.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+class GpuBlock:
+    """One layer on the GPU plus its workspace, driven through the C ABI."""
+
+    def __init__(self, layer, max_tokens: int):
+        self.layer = layer
+        self.L = moe.make_layer_struct(layer)
+        self.ws = moe.alloc_workspace(self.L, max_tokens)
+        self.sh = layer.shape
+
+    def route(self, x, flags=0):
+        T = x.shape[0]
+        logits = torch.empty(T, self.sh.E, dtype=torch.float32, device="cuda")
+        ids = torch.empty(T, self.sh.k, dtype=torch.int32, device="cuda")
+        w = torch.empty(T, self.sh.k, dtype=torch.float32, device="cuda")
+        moe.moe_route_topk(self.L, x, T, flags, logits, ids, w, self.ws)
+        return logits, ids, w
+
+    def decode(self, x, ids, w, flags=0):
+        y = torch.empty_like(x)
+        moe.moe_expert_ffn_decode(self.L, x, x.shape[0], ids, w, y, flags, self.ws)
+        return y
+
+    def prefill(self, x, ids, w, flags=0, want_buckets=False):
+        T = x.shape[0]
+        y = torch.empty_like(x)
+        off = ent = None
+        if want_buckets:
+            off = torch.empty(self.sh.E + 1, dtype=torch.int32, device="cuda")
+            ent = torch.empty(T * self.sh.k, dtype=torch.int32, device="cuda")
+        moe.moe_expert_ffn_prefill(self.L, x, T, ids, w, y, off, ent, flags, self.ws)
+        return (y, off, ent) if want_buckets else y
+
+    def block(self, x, flags=0):
+        y = torch.empty_like(x)
+        moe.moe_block_forward(self.L, x, x.shape[0], y, flags, self.ws)
+        return y
+
+    def error_word(self):
+        return moe.moe_workspace_error(self.ws)
+
+
+def oracle_check(layer, x, logits, ids, w, y, flags=0, rows=None, oflags=None):
+    """Compare one GPU block result with the oracle (selection on the GPU's
+    fp32 logits).  Returns (max rel, rms rel)."""
+    OL = oracle.OracleLayer(layer.to("cpu") if layer.codes.is_cuda else layer)
+    of = 0
+    if flags & moe.F_PRENORM:
+        of |= oracle.PRENORM
+    if flags & moe.F_RESIDUAL:
+        of |= oracle.RESIDUAL
+    lg = logits.cpu().numpy()
+    r = OL.block_forward(bf16_bits(x), rows=rows, sel_logits=lg, flags=of)
+    rr = np.arange(x.shape[0]) if rows is None else np.asarray(rows)
+    ids_g = ids.cpu().numpy()[rr]
+    assert np.array_equal(ids_g, r["ids"]), "routing differs from the oracle's selection"
+    # logits within the fp32 bound of the oracle's fp64 logits
+    if flags & moe.F_PRENORM:
+        xin = oracle.rmsnorm_bf16(bf16_bits(x)[rr])
+        xin = torch.from_numpy(xin.view(np.int16)).view(torch.bfloat16).double().numpy()
+    else:
+        xin = x.cpu().double().numpy()[rr]
+    bound = logit_bound(layer, xin)
+    assert np.all(np.abs(lg[rr] - r["logits"]) <= bound), "router logits outside the fp32 bound"
+    wg = w.cpu().double().numpy()[rr]
+    assert np.allclose(wg, r["w"], rtol=1e-5, atol=1e-6), "routing weights differ"
+    assert np.allclose(wg.sum(1), 1.0, atol=1e-6)
+    yg = y.float().cpu().double().numpy()[rr]
+    return assert_close(yg, r["y"])

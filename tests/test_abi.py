@@ -1,0 +1,110 @@
+"""The C ABI library: it loads, exports every entry point include/moe.h
+declares, and its host-side validation answers before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from routed_expert_ffn_06_b200 import build, moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return moe.load()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ["moe_route_topk", "moe_expert_ffn_decode", "moe_expert_ffn_prefill",
+              "moe_block_forward", "moe_workspace_bytes"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in _declared():
+        assert hasattr(lib, n), f"{n} declared in include/moe.h but not exported"
+    assert set(_declared()) <= set(moe.EXPORTS) | set(_declared())
+
+
+def _layer(**kw):
+    base = dict(d_model=64, n_experts=16, ffn=32, top_k=2, bits=2, group=32, shared_ffn=32)
+    base.update(kw)
+    L = moe.moe_layer(**base)
+    fake = 0x7F0000000000  # 256-aligned fake device addresses: never dereferenced on the host
+    L.router_w = fake
+    L.expert_slot = fake + 0x1000
+    L.codes = fake + 0x2000
+    L.scales = fake + 0x100000
+    L.shared_codes = fake + 0x200000
+    L.shared_scales = fake + 0x300000
+    return L
+
+
+def test_workspace_bytes(lib):
+    L = _layer()
+    n1 = moe.moe_workspace_bytes(L, 1)
+    n4 = moe.moe_workspace_bytes(L, 4)
+    n8k = moe.moe_workspace_bytes(L, 8192)
+    assert 0 < n1 <= n4 < n8k
+    assert n8k % 256 == 0
+    assert moe.moe_workspace_bytes(_layer(bits=4), 4) == 0
+    assert moe.moe_workspace_bytes(_layer(d_model=48), 4) == 0
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(bits=4), 2), (dict(group=64), 2), (dict(d_model=48), 2), (dict(ffn=40), 2),
+    (dict(top_k=17), 2), (dict(top_k=0), 2), (dict(n_experts=1), 2), (dict(n_experts=2048), 2),
+    (dict(shared_ffn=-32), 2), (dict(d_model=8192), 2),
+])
+def test_shape_validation(lib, bad, status):
+    L = _layer(**bad)
+    rc = lib.moe_block_forward(ctypes.byref(L), 0x7F0000400000, 4, 0x7F0000500000, 0,
+                               0x7F0000600000, 1 << 30, None)
+    assert rc == status
+
+
+def test_pointer_and_size_validation(lib):
+    L = _layer()
+    ws, x, y = 0x7F0000600000, 0x7F0000400000, 0x7F0000500000
+    P = ctypes.byref
+    assert lib.moe_block_forward(P(L), None, 4, y, 0, ws, 1 << 30, None) == 1
+    assert lib.moe_block_forward(P(L), x, -1, y, 0, ws, 1 << 30, None) == 1
+    assert lib.moe_block_forward(P(L), x + 2, 4, y, 0, ws, 1 << 30, None) == 4     # misaligned x
+    assert lib.moe_block_forward(P(L), x, 4, y, 0, ws + 16, 1 << 30, None) == 4    # ws not 256-aligned
+    assert lib.moe_block_forward(P(L), x, 4, y, 0, ws, 64, None) == 3              # too small
+    assert lib.moe_expert_ffn_decode(P(L), x, 9, x, x, y, 0, ws, 1 << 30, None) == 2  # T > 8
+    assert lib.moe_expert_ffn_decode(P(L), x, 4, x, x, x, 0, ws, 1 << 30, None) == 1  # y aliases x
+    assert lib.moe_route_topk(P(L), x, 4, 1 << 7, None, x, x, ws, 1 << 30, None) == 1  # bad flag
+    L2 = _layer()
+    L2.codes = 0x7F0000002008
+    assert lib.moe_block_forward(P(L2), x, 4, y, 0, ws, 1 << 30, None) == 4
+    L3 = _layer()
+    L3.shared_codes = None
+    assert lib.moe_block_forward(P(L3), x, 4, y, 0, ws, 1 << 30, None) == 1
+    assert lib.moe_block_forward(None, x, 4, y, 0, ws, 1 << 30, None) == 1
+
+
+def test_no_gpu_reports_no_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    L = _layer()
+    rc = lib.moe_block_forward(ctypes.byref(L), 0x7F0000400000, 4, 0x7F0000500000, 0,
+                               0x7F0000600000, 1 << 30, None)
+    assert rc == 8
+
+
+def test_status_strings(lib):
+    assert moe.moe_status_string(0) == "ok"
+    assert "workspace" in moe.moe_status_string(3)
+    assert "sm_100a" in moe.moe_build_info()

@@ -1,0 +1,152 @@
+"""GPU parity of the router and the decode / verify-window step against the
+fp64 oracle, through the C ABI.  Routing must match bit for bit given the
+device's fp32 logits; outputs within max rel 2e-2 / RMS rel 3e-3."""
+import numpy as np
+import pytest
+import torch
+
+from routed_expert_ffn_06_b200 import build, moe, synth
+from _util import GpuBlock, assert_close, errors, oracle_check
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    moe.load()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def _layer(shape, **kw):
+    kw.setdefault("bias", "normal")
+    return synth.make_layer(shape, device="cuda", **kw)
+
+
+# -------------------------------------------------------------- tiny config
+def test_tiny_config_block():
+    """d=64, 16 experts (ffn 32) + shared (ffn 32), top-2, 4 tokens, 2-bit, seed 0."""
+    wl = synth.WORKLOADS["tiny"]
+    layer = synth.make_layer(wl["shape"], seed=0, device="cuda", bias=wl["bias"], slot=wl["slot"])
+    x = synth.make_tokens(4, 64, seed=0, device="cuda")
+    gb = GpuBlock(layer, 8)
+    logits, ids, w = gb.route(x)
+    y = gb.decode(x, ids, w)
+    oracle_check(layer, x, logits, ids, w, y)
+    y2 = gb.block(x)
+    assert torch.equal(y, y2)
+    assert gb.error_word() == (0, 0)
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("E,k,Fs", [(16, 2, 32), (37, 5, 0), (64, 16, 64), (8, 8, 32)])
+def test_small_shapes(bits, T, E, k, Fs):
+    sh = synth.MoEShape(d=96, E=E, F=64, Fs=Fs, k=k, bits=bits)
+    layer = _layer(sh, seed=T * 7 + E, bias_std=1.0)
+    x = synth.make_tokens(T, 96, seed=T, device="cuda")
+    gb = GpuBlock(layer, 8)
+    logits, ids, w = gb.route(x)
+    y = gb.decode(x, ids, w)
+    oracle_check(layer, x, logits, ids, w, y)
+    assert gb.error_word() == (0, 0)
+
+
+@pytest.mark.parametrize("flags", [moe.F_PRENORM, moe.F_RESIDUAL, moe.F_PRENORM | moe.F_RESIDUAL])
+def test_flags_small(flags):
+    sh = synth.MoEShape(d=128, E=32, F=64, Fs=64, k=4, bits=3)
+    layer = _layer(sh, seed=3)
+    x = (synth.make_tokens(4, 128, seed=9, device="cuda").float() * 3.0).to(torch.bfloat16)
+    gb = GpuBlock(layer, 8)
+    logits, ids, w = gb.route(x, flags)
+    y = gb.decode(x, ids, w, flags)
+    oracle_check(layer, x, logits, ids, w, y, flags=flags)
+
+
+def test_zero_tokens_is_a_noop():
+    sh = synth.MoEShape(d=64, E=16, F=32, Fs=32, k=2, bits=2)
+    gb = GpuBlock(_layer(sh), 4)
+    x = torch.ones(1, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((1, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_block_forward(gb.L, x, 0, y, 0, gb.ws)
+    torch.cuda.synchronize()
+    assert torch.all(y == 7.0)
+
+
+def test_zero_input_gives_zero():
+    sh = synth.MoEShape(d=128, E=32, F=64, Fs=64, k=4, bits=2)
+    gb = GpuBlock(_layer(sh), 4)
+    x = torch.zeros(4, 128, dtype=torch.bfloat16, device="cuda")
+    assert torch.count_nonzero(gb.block(x)) == 0
+
+
+def test_out_of_range_ids_are_flagged_not_read():
+    sh = synth.MoEShape(d=64, E=16, F=32, Fs=32, k=2, bits=2)
+    layer = _layer(sh)
+    gb = GpuBlock(layer, 4)
+    x = synth.make_tokens(2, 64, device="cuda")
+    ids = torch.tensor([[3, 99], [-1, 5]], dtype=torch.int32, device="cuda")
+    w = torch.full((2, 2), 0.5, dtype=torch.float32, device="cuda")
+    gb.decode(x, ids, w)
+    st, code = gb.error_word()
+    assert st == 6 and code & 2
+    assert gb.error_word() == (0, 0)      # the read clears it
+
+
+# --------------------------------------------------------------- full size
+@pytest.fixture(scope="module")
+def decode_layer():
+    wl = synth.WORKLOADS["decode"]
+    return synth.make_layer(wl["shape"], seed=0, device="cuda", bias=wl["bias"], slot=wl["slot"])
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 4])
+def test_decode_full_size(decode_layer, T):
+    """d=2048, 512 experts ffn 512 + shared, top-10, 2-bit, Zipf(1.1) popularity."""
+    gb = GpuBlock(decode_layer, 8)
+    x = synth.make_tokens(T, 2048, seed=100 + T, device="cuda")
+    logits, ids, w = gb.route(x)
+    y = gb.decode(x, ids, w)
+    mr, rr = oracle_check(decode_layer, x, logits, ids, w, y)
+    print(f"T={T}: max rel {mr:.2e} rms rel {rr:.2e}")
+    assert gb.error_word() == (0, 0)
+
+
+def test_decode_window_invariance(decode_layer):
+    """A verify window gives each token what it gets alone: same routing,
+    outputs equal within tolerance."""
+    gb = GpuBlock(decode_layer, 8)
+    x = synth.make_tokens(4, 2048, seed=55, device="cuda")
+    _, ids4, w4 = gb.route(x)
+    y4 = gb.decode(x, ids4, w4)
+    for t in range(4):
+        _, ids1, w1 = gb.route(x[t:t + 1])
+        y1 = gb.decode(x[t:t + 1].clone(), ids1, w1)
+        assert torch.equal(ids1[0], ids4[t])
+        assert_close(y4[t:t + 1].float().cpu().double().numpy(), y1.float().cpu().double().numpy(),
+                     max_rel=1e-2, rms_rel=3e-3)
+
+
+def test_decode_slot_layout_invariance():
+    """The same experts packed into other slots: bit-identical output."""
+    sh = synth.MoEShape(d=512, E=64, F=128, Fs=128, k=6, bits=3)
+    a = synth.make_layer(sh, seed=4, device="cuda", bias="normal", slot="identity")
+    b = synth.make_layer(sh, seed=4, device="cuda", bias="normal", slot="random")
+    assert not torch.equal(a.expert_slot, b.expert_slot)
+    x = synth.make_tokens(4, 512, seed=8, device="cuda")
+    ya = GpuBlock(a, 4).block(x)
+    yb = GpuBlock(b, 4).block(x)
+    assert torch.equal(ya, yb)
+
+
+def test_decode_3bit_stack_layer_prenorm_residual():
+    """One layer of the 48-layer 3-bit stack, with pre-norm and residual."""
+    wl = synth.WORKLOADS["decode_stack"]
+    layer = synth.make_layer(wl["shape"], seed=0, layer=7, device="cuda", bias=wl["bias"],
+                             slot=wl["slot"])
+    gb = GpuBlock(layer, 4)
+    x = (synth.make_tokens(4, 2048, seed=7, device="cuda").float() * 20).to(torch.bfloat16)
+    flags = moe.F_PRENORM | moe.F_RESIDUAL
+    logits, ids, w = gb.route(x, flags)
+    y = gb.decode(x, ids, w, flags)
+    oracle_check(layer, x, logits, ids, w, y, flags=flags)
