@@ -1,0 +1,407 @@
+"""Benchmark of the routed sparse-MoE block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|stack]
+                    [--impl ours|reference]
+
+Default workload (the configuration the headline metric is quoted on): one
+routed-MoE layer, d=2048, 512 experts (SwiGLU ffn 512) + shared expert, top-10,
+2-bit group-32 weights with fp16 scales, Zipf(1.1) popularity, frequency-ordered
+slots; verify windows of T = 1, 2, 3 and 4 tokens.  A step is one pass of the
+block (router, top-k, expert FFNs, shared expert, combine) over each of the four
+windows, each on another of 32 independent layer copies (16 GB of weights, far
+above the 126 MB L2), with fresh tokens.  Steps are captured in a CUDA graph and
+replayed; the timed region is bracketed by a barrier and device syncs, timed with
+CUDA events, max over ranks.  One process per GPU; ranks run independent replicas
+(no collective on the data path).
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("routed-MoE tokens/s (decode 1–4 tok, 8192 prefill); HBM GB/s & TC util vs peak")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=None)
+    p.add_argument("--warmup", type=int, default=None)
+    p.add_argument("--workload", default="decode", choices=["decode", "prefill", "stack"])
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--layers", type=int, default=32, help="independent layer copies rotated")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------- plumbing
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200",
+                                       "-i", str(self.dev)], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+
+    def summary(self):
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as f:
+            for line in f:
+                parts = [s.strip() for s in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d["bf16_tflops_sustained"]), "src": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "src": "fallback"}
+
+
+# ------------------------------------------------------------------ decode
+DECODE_WINDOWS = (1, 2, 3, 4)
+
+
+def expert_bytes(shape) -> int:
+    from routed_expert_ffn_06_b200 import synth
+    return shape.codes_bytes + shape.n_scales * 2
+
+
+def oracle_cpu_baseline(layer_cpu, windows, seconds, seed=777):
+    """The oracle, as it stands, on this host's cores: whole windows until
+    `seconds` of CPU work have run.  Returns (tokens/s, cores, sample)."""
+    import oracle
+    from routed_expert_ffn_06_b200 import synth
+    OL = oracle.OracleLayer(layer_cpu)
+    toks, t0, n_win = 0, time.perf_counter(), 0
+    while time.perf_counter() - t0 < seconds:
+        for T in windows:
+            x = synth.make_tokens(T, layer_cpu.shape.d, seed=seed, step=n_win)
+            OL.block_forward(x)
+            toks += T
+            n_win += 1
+    dt = time.perf_counter() - t0
+    return toks / dt, oracle.num_threads(), f"{n_win} windows ({toks} tokens, T cycling {windows})"
+
+
+def bench_decode(args, rank, world, local):
+    import torch
+
+    from routed_expert_ffn_06_b200 import moe, synth
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    moe.load()
+    wl = synth.WORKLOADS["decode"]
+    sh = wl["shape"]
+    NL = args.layers
+    K = args.steps if args.steps is not None else 20000
+    W = args.warmup if args.warmup is not None else 200
+    G = 500                      # steps per captured graph
+    t_gen = time.time()
+    layers = [synth.make_layer(sh, seed=rank * 1000 + i, layer=i, device=dev, bias=wl["bias"],
+                               slot=wl["slot"]) for i in range(NL)]
+    t_gen = time.time() - t_gen
+    structs = [moe.make_layer_struct(l) for l in layers]
+    ws = moe.alloc_workspace(structs[0], max(DECODE_WINDOWS))
+    nwin = len(DECODE_WINDOWS)
+    ntok_step = sum(DECODE_WINDOWS)
+    # fresh tokens per step (G distinct steps per graph)
+    xs = [[synth.make_tokens(T, sh.d, seed=rank * 1000 + 7, step=s * nwin + i, device=dev)
+           for i, T in enumerate(DECODE_WINDOWS)] for s in range(G)]
+    ys = [torch.empty(max(DECODE_WINDOWS), sh.d, dtype=torch.bfloat16, device=dev)
+          for _ in range(nwin)]
+    ids = [[torch.empty(T, sh.k, dtype=torch.int32, device=dev) for T in DECODE_WINDOWS]
+           for _ in range(G)]
+    wts = [[torch.empty(T, sh.k, dtype=torch.float32, device=dev) for T in DECODE_WINDOWS]
+           for _ in range(G)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def enqueue_step(s, events=None):
+        for i, T in enumerate(DECODE_WINDOWS):
+            L = structs[(s * nwin + i) % NL]
+            moe.moe_route_topk(L, xs[s][i], T, 0, None, ids[s][i], wts[s][i], ws, stream)
+            if events is not None:
+                events[s][i][0].record(stream)
+            moe.moe_expert_ffn_decode(L, xs[s][i], T, ids[s][i], wts[s][i], ys[i], 0, ws, stream)
+            if events is not None:
+                events[s][i][1].record(stream)
+
+    # eager pass: sets kernel attributes, fills routing for the byte counts
+    with torch.cuda.stream(stream):
+        for s in range(G):
+            enqueue_step(s)
+    stream.synchronize()
+    st, code = moe.moe_workspace_error(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device error word {code:#x}")
+    # algorithmic bytes of every expert step: unique experts of the window + shared
+    eb = expert_bytes(sh)
+    step_expert_bytes = []
+    for s in range(G):
+        tot = 0
+        for i, T in enumerate(DECODE_WINDOWS):
+            U = int(torch.unique(ids[s][i]).numel())
+            tot += (U + 1) * eb + 2 * T * sh.d * 2
+        step_expert_bytes.append(tot)
+
+    # graphs: one of G steps
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for s in range(G):
+            enqueue_step(s)
+    reps_w = max(1, W // G)
+    reps = max(1, K // G)
+    K = reps * G
+    W = reps_w * G
+    with torch.cuda.stream(stream):
+        for _ in range(reps_w):
+            g.replay()
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(ms, world)
+    clocks = clk.summary()
+    value = K * ntok_step * world / (ms / 1e3)
+
+    # component timing (same workload, events around each expert step)
+    Gc = min(G, 200)
+    # external events: recorded as event nodes inside the graph, timed at replay
+    evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+            for _ in DECODE_WINDOWS] for _ in range(Gc)]
+    gc = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gc, stream=stream):
+        for s in range(Gc):
+            enqueue_step(s, evs)
+    with torch.cuda.stream(stream):
+        gc.replay()
+    stream.synchronize()
+    exp_ms = [evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(Gc)
+              for i in range(nwin)]
+    exp_bytes = sum(step_expert_bytes[:Gc])
+    achieved = exp_bytes / (sum(exp_ms) / 1e3) / 1e9
+    per_T = {}
+    for i, T in enumerate(DECODE_WINDOWS):
+        tms = [evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(Gc)]
+        per_T[str(T)] = round(1e3 * sum(tms) / len(tms), 2)
+    peaks = measured_peaks()
+
+    # end to end through the public call with host buffers
+    Ke = min(K, 2000)
+    xh = [[x.cpu().pin_memory() for x in xs[s]] for s in range(G)]
+    yh = [torch.empty(T, sh.d, dtype=torch.bfloat16).pin_memory() for T in DECODE_WINDOWS]
+    xd = [torch.empty(T, sh.d, dtype=torch.bfloat16, device=dev) for T in DECODE_WINDOWS]
+    ysd = [torch.empty(T, sh.d, dtype=torch.bfloat16, device=dev) for T in DECODE_WINDOWS]
+    barrier(world)
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for s in range(Ke):
+            for i, T in enumerate(DECODE_WINDOWS):
+                L = structs[(s * nwin + i) % NL]
+                xd[i].copy_(xh[s % G][i], non_blocking=True)
+                moe.moe_block_forward(L, xd[i], T, ysd[i], 0, ws, stream)
+                yh[i].copy_(ysd[i], non_blocking=True)
+        f1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
+    e2e_value = Ke * ntok_step * world / (e2e_ms / 1e3)
+
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic (seeded; random-init weights of the stated architecture)",
+        "config": {"workload": "decode single layer: d=2048, 512 experts ffn=512 + shared "
+                               "ffn=512, top-10, 2-bit g32 fp16 scales, Zipf(1.1) popularity, "
+                               "frequency-ordered slots; windows T=1,2,3,4 per step",
+                   "tokens_per_step": ntok_step, "layer_copies": NL,
+                   "l2": "inputs larger than L2 (32 layer copies rotated, "
+                         f"{NL * (sh.E * eb + sh.E * sh.d * 4) / 1e9:.1f} GB)",
+                   "parallelism": f"replicas x{world}", "graph_steps": G,
+                   "mma": "f16 x f16 -> f32 (weights dequantised in registers)",
+                   "weights_gen_s": round(t_gen, 1)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": None, "peak_src": peaks["src"],
+                     "kernel": "expert step (decode_gu + decode_dn per moe_expert_ffn_decode call)",
+                     "bytes_per_launch": round(exp_bytes / (Gc * nwin)),
+                     "us_per_launch_by_T": per_T},
+        "clocks": clocks,
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": ntok_step * sh.d * 2, "d2h_bytes_per_step": ntok_step * sh.d * 2,
+                "steps": Ke, "path": "moe_block_forward via the ctypes binding, pinned host x/y"},
+        "gpu_launches": K * nwin * 3,   # router, gate/up, down per window
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = oracle_cpu_baseline(layers[0].to("cpu"), DECODE_WINDOWS,
+                                               args.cpu_seconds)
+        res["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cores,
+                               "kind": "oracle", "sample": sample}
+    return res
+
+
+# --------------------------------------------------------------- reference
+def run_reference(args, rank, world):
+    """The fp64 oracle on the host cores, same workload and metric."""
+    if rank != 0:
+        return None
+    import oracle
+    from routed_expert_ffn_06_b200 import synth
+    wl = synth.WORKLOADS["decode"]
+    layer = synth.make_layer(wl["shape"], seed=0, device="cpu", bias=wl["bias"], slot=wl["slot"])
+    OL = oracle.OracleLayer(layer)
+    K = args.steps if args.steps is not None else 5
+    W = args.warmup if args.warmup is not None else 1
+    W = min(W, 3)
+    K = min(K, 20)
+
+    def step(s):
+        for i, T in enumerate(DECODE_WINDOWS):
+            OL.block_forward(synth.make_tokens(T, wl["shape"].d, seed=7, step=s * 4 + i))
+    for s in range(W):
+        step(s)
+    t0 = time.perf_counter()
+    for s in range(K):
+        step(W + s)
+    dt = time.perf_counter() - t0
+    v = K * sum(DECODE_WINDOWS) / dt
+    return {"metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": round(1e3 * dt / K, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "decode single layer: d=2048, 512 experts ffn=512 + shared, "
+                                   "top-10, 2-bit g32, Zipf(1.1); windows T=1,2,3,4 per step"},
+            "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": f"{K} steps of 4 windows (10 tokens)"},
+            "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_init()
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, rank, world)
+        elif args.workload == "decode":
+            res = bench_decode(args, rank, world, local)
+        elif args.workload == "prefill":
+            from routed_expert_ffn_06_b200 import benchlib
+            res = benchlib.bench_prefill(args, rank, world, local)
+        else:
+            from routed_expert_ffn_06_b200 import benchlib
+            res = benchlib.bench_stack(args, rank, world, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -122,9 +122,10 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 
 // -------------------------------------------------------------- mma.sync
 // D(16x8 f32) = A(16x16 f16, row) * B(16x8 f16, col) + C
+// Not volatile: the compiler may interleave independent MMAs and their loads.
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4],
                                               const uint32_t (&b)[2], const float (&c)[4]) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])

@@ -20,47 +20,65 @@ constexpr float kRmsEps = 1e-6f;
 
 // ---------------------------------------------------------------- selection
 // One warp selects top_k of E (E <= 1024) logits of one token and writes the
-// ids (largest first) and renormalised weights.
+// ids (largest first) and renormalised weights.  Each lane keeps the best of
+// its own logits (ties: lowest index, as the lane scans upward); a round takes
+// the warp maximum of the keys and the lowest index holding it (two redux
+// instructions), and only the winning lane rescans.
 __device__ void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
                           float* __restrict__ w, Control* ctl, bool debug) {
   const int lane = threadIdx.x & 31;
-  uint32_t key[32];
-  uint32_t taken = 0;
+  // all loads first (independent, in flight together), checks afterwards
+  float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    int e = lane + 32 * i;
-    key[i] = 0u;
-    if (e < E) {
-      float v = __ldcg(row + e);
-      if (debug && !isfinite(v)) record_error(ctl, kErrNonFinite, 0x100);
-      key[i] = order_key(v);
-    }
+    const int e = lane + 32 * i;
+    v[i] = e < E ? __ldcg(row + e) : 0.f;
   }
-  float my_v = 0.f;
-  for (int j = 0; j < k; ++j) {
-    // lane-local best: larger key, then lower index (lower i within a lane)
-    unsigned long long best = 0ull;
+  uint32_t key[32];
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    key[i] = order_key(v[i]);
+    bad |= (lane + 32 * i < E) && !isfinite(v[i]);
+  }
+  if (debug && bad) record_error(ctl, kErrNonFinite, 0x100);
+  uint32_t taken = 0;
+  // lane-local best by a depth-5 tree over (key << 32 | ~index): larger key
+  // wins, equal keys go to the lower index; 0 marks invalid or taken entries
+  uint32_t bk = 0u, bi = 0xFFFFFFFFu;
+  auto rescan = [&]() {
+    unsigned long long c[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u)) {
-        unsigned long long c = (static_cast<unsigned long long>(key[i]) << 32) |
-                               static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(e));
-        best = c > best ? c : best;
-      }
+      const uint32_t e = (uint32_t)(lane + 32 * i);
+      const bool ok = ((int)e < E) && !((taken >> i) & 1u);
+      c[i] = ok ? ((unsigned long long)key[i] << 32) | (unsigned long long)(~e) : 0ull;
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-      best = other > best ? other : best;
+    for (int half = 16; half >= 1; half >>= 1) {
+#pragma unroll
+      for (int i = 0; i < half; ++i) c[i] = c[i + half] > c[i] ? c[i + half] : c[i];
     }
-    const uint32_t e = 0xFFFFFFFFu - static_cast<uint32_t>(best & 0xFFFFFFFFull);
-    const uint32_t kk = static_cast<uint32_t>(best >> 32);
-    if ((int)(e & 31u) == lane) taken |= 1u << (e >> 5);
-    uint32_t u = (kk & 0x80000000u) ? (kk & 0x7FFFFFFFu) : ~kk;
-    const float v = __uint_as_float(u);
-    if (lane == j) my_v = v;
-    if (lane == 0) ids[j] = static_cast<int32_t>(e);
+    if (c[0] == 0ull) {
+      bk = 0u;
+      bi = 0xFFFFFFFFu;
+    } else {
+      bk = (uint32_t)(c[0] >> 32);
+      bi = ~(uint32_t)(c[0] & 0xFFFFFFFFull);
+    }
+  };
+  rescan();
+  float my_v = 0.f;
+  for (int j = 0; j < k; ++j) {
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, bi == 0xFFFFFFFFu ? 0u : bk);
+    const uint32_t win = __reduce_min_sync(0xffffffffu, (bi != 0xFFFFFFFFu && bk == mk) ? bi : 0xFFFFFFFFu);
+    const uint32_t u = (mk & 0x80000000u) ? (mk & 0x7FFFFFFFu) : ~mk;
+    if (lane == j) my_v = __uint_as_float(u);
+    if (lane == 0) ids[j] = static_cast<int32_t>(win);
+    if ((win & 31u) == (uint32_t)lane) {
+      taken |= 1u << (win >> 5);
+      rescan();
+    }
   }
   const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
   const float ex = lane < k ? expf(my_v - v0) : 0.f;
@@ -69,74 +87,86 @@ __device__ void warp_topk(const float* __restrict__ row, int E, int k, int32_t* 
 }
 
 // --------------------------------------------------------- x (bf16) staging
-// Loads T token rows into shared memory as bf16 bits; with PRENORM replaces
-// them by bf16(x / sqrt(mean(x^2) + eps)), computed in fp32.
+// Loads T token rows into shared memory as bf16 bits (16-byte loads, all
+// tokens in one pass); with PRENORM replaces them by
+// bf16(x / sqrt(mean(x^2) + eps)), computed in fp32.  red: >= T floats.
 __device__ void stage_tokens(const uint16_t* __restrict__ x, int T, int d, bool prenorm,
                              uint16_t* xs, float* red) {
   const int tid = threadIdx.x, nt = blockDim.x;
-  const int nw = nt / 32;
-  for (int t = 0; t < T; ++t) {
-    const uint16_t* xr = x + (size_t)t * d;
-    float ss = 0.f;
-    for (int i = tid; i < d; i += nt) {
-      uint16_t b = xr[i];
-      xs[t * d + i] = b;
-      float v = bf16_bits_to_float(b);
-      ss += v * v;
-    }
+  if (prenorm) {
+    for (int t = tid; t < T; t += nt) red[t] = 0.f;
+    __syncthreads();
+  }
+  const int per = d / 8;
+  for (int i = tid; i < T * per; i += nt) {
+    const uint4 v = reinterpret_cast<const uint4*>(x)[i];
+    reinterpret_cast<uint4*>(xs)[i] = v;
     if (prenorm) {
-      ss = warp_sum(ss);
-      if ((tid & 31) == 0) red[tid >> 5] = ss;
-      __syncthreads();
-      float tot = 0.f;
-      for (int i = 0; i < nw; ++i) tot += red[i];
-      const float inv = rsqrtf(tot / (float)d + kRmsEps);
-      for (int i = tid; i < d; i += nt) {
-        float v = bf16_bits_to_float(xs[t * d + i]) * inv;
-        __nv_bfloat16 bv = __float2bfloat16_rn(v);
-        xs[t * d + i] = *reinterpret_cast<uint16_t*>(&bv);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      float ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float a = __uint_as_float(w4[j] << 16), b = __uint_as_float(w4[j] & 0xFFFF0000u);
+        ss += a * a + b * b;
       }
-      __syncthreads();
+      atomicAdd(&red[i / per], ss);
     }
   }
   __syncthreads();
+  if (prenorm) {
+    for (int i = tid; i < T * d; i += nt) {
+      const float inv = rsqrtf(red[i / d] / (float)d + kRmsEps);
+      __nv_bfloat16 bv = __float2bfloat16_rn(bf16_bits_to_float(xs[i]) * inv);
+      xs[i] = *reinterpret_cast<uint16_t*>(&bv);
+    }
+    __syncthreads();
+  }
 }
 
 // ------------------------------------------------------------- small T router
-// grid: ceil(E/4) CTAs of 4 warps, one warp per expert row.
-// smem: T*d bf16 + 32 floats.
-__global__ void __launch_bounds__(128) router_small_kernel(LayerDev L, const uint16_t* __restrict__ x,
-                                                           int T, uint32_t flags,
-                                                           float* __restrict__ logits,
-                                                           int32_t* __restrict__ ids,
-                                                           float* __restrict__ wout, Control* ctl) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
-  float* red = reinterpret_cast<float*>(smem + ((size_t)T * L.d * 2 + 15) / 16 * 16);
+// grid: ceil(E/4) CTAs of 16 warps; four warps per expert row, each a quarter
+// of d.  The CTA's four rows of Wr (contiguous) are requested with one bulk
+// async copy before the grid waits on its predecessor (Wr depends on nothing
+// earlier), so the whole 4 MiB router is in flight at once.  The last CTA to
+// finish (atomic counter in the workspace, reset by that CTA) selects.
+// smem: 4*d fp32 (rows) | T*d bf16 (tokens) | 4*4*8 partial sums.
+constexpr int kRouterRows = 4;
+constexpr int kRouterWarps = 16;
+__global__ void __launch_bounds__(kRouterWarps * 32) router_small_kernel(
+    LayerDev L, const uint16_t* __restrict__ x, int T, uint32_t flags, float* __restrict__ logits,
+    int32_t* __restrict__ ids, float* __restrict__ wout, Control* ctl) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  float* wrs = reinterpret_cast<float*>(smem);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + (size_t)kRouterRows * L.d * 4);
+  __shared__ float red[kMaxDecodeT];
+  __shared__ float part[kRouterRows][4][kMaxDecodeT];
   __shared__ int s_last;
+  __shared__ __align__(8) uint64_t bar;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * 4 + warp;
-
-  // Wr does not depend on earlier kernels: pull this warp's row into L2 first.
-  if (e < L.E && lane == 0) {
-    const char* row = reinterpret_cast<const char*>(L.Wr + (size_t)e * L.d);
-    for (int off = 0; off < L.d * 4; off += 4096) {
-      int n = min(4096, L.d * 4 - off);
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(row + off), "r"(n) : "memory");
-    }
+  const int e0 = blockIdx.x * kRouterRows;
+  const int nrows = min(kRouterRows, L.E - e0);
+  const int row = warp >> 2, quarter = warp & 3;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    const uint32_t bytes = (uint32_t)nrows * L.d * 4;
+    mbar_arrive_expect_tx(&bar, bytes);
+    bulk_g2s(wrs, L.Wr + (size_t)e0 * L.d, bytes, &bar);
   }
   pdl_wait();
   pdl_launch_dependents();
-  stage_tokens(x, T, L.d, flags & MOE_F_PRENORM, xs, red);
+  stage_tokens(x, T, L.d, flags & MOE_F_PRENORM, xs, red);   // ends with __syncthreads
+  const bool have = mbar_wait(&bar, 0, ctl, 0x110);
 
-  if (e < L.E) {
+  if (row < nrows && have) {
     float acc[kMaxDecodeT];
 #pragma unroll
     for (int t = 0; t < kMaxDecodeT; ++t) acc[t] = 0.f;
-    const float4* wr = reinterpret_cast<const float4*>(L.Wr + (size_t)e * L.d);
-    const int nc = L.d / 4;
-    for (int c = lane; c < nc; c += 32) {
-      const float4 wv = __ldg(wr + c);
+    const float4* wr = reinterpret_cast<const float4*>(wrs + (size_t)row * L.d);
+    const int nc = L.d / 4, c0 = quarter * (nc / 4), c1 = c0 + nc / 4;
+#pragma unroll 4
+    for (int c = c0 + lane; c < c1; c += 32) {
+      const float4 wv = wr[c];
 #pragma unroll
       for (int t = 0; t < kMaxDecodeT; ++t) {
         if (t < T) {
@@ -148,43 +178,49 @@ __global__ void __launch_bounds__(128) router_small_kernel(LayerDev L, const uin
         }
       }
     }
-    const float b = L.bias ? L.bias[e] : 0.f;
 #pragma unroll
     for (int t = 0; t < kMaxDecodeT; ++t) {
       if (t < T) {
-        float s = warp_sum(acc[t]);
-        if (lane == 0) logits[(size_t)t * L.E + e] = s + b;
+        const float s = warp_sum(acc[t]);
+        if (lane == 0) part[row][quarter][t] = s;
       }
     }
   }
   __syncthreads();
+  if (threadIdx.x < nrows * T) {
+    const int r = threadIdx.x / T, t = threadIdx.x % T, e = e0 + r;
+    const float s = part[r][0][t] + part[r][1][t] + part[r][2][t] + part[r][3][t];
+    logits[(size_t)t * L.E + e] = s + (L.bias ? L.bias[e] : 0.f);
+  }
+  __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
+    __threadfence();   // release this CTA's logits
     const uint32_t old = atomicAdd(&ctl->router_done, 1u);
     s_last = (old == gridDim.x - 1);
+    if (s_last) __threadfence();   // acquire every CTA's logits; the barrier below publishes
   }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
-  for (int t = warp; t < T; t += 4)
+  for (int t = warp; t < T; t += kRouterWarps)
     warp_topk(logits + (size_t)t * L.E, L.E, L.k, ids + (size_t)t * L.k, wout + (size_t)t * L.k,
               ctl, flags & MOE_F_DEBUG);
   if (threadIdx.x == 0) atomicExch(&ctl->router_done, 0u);
 }
 
+size_t router_small_smem(int d, int T) {
+  return (size_t)kRouterRows * d * 4 + ((size_t)T * d * 2 + 15) / 16 * 16;
+}
+
 cudaError_t launch_router_small(const LayerDev& L, const uint16_t* x, int T, uint32_t flags,
                                 float* logits, int32_t* ids, float* w, Control* ctl,
                                 cudaStream_t st) {
-  size_t smem = ((size_t)T * L.d * 2 + 15) / 16 * 16 + 32 * sizeof(float);
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaFuncSetAttribute(router_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         96 * 1024);
-    attr_done = true;
-  }
-  dim3 grid((L.E + 3) / 4);
-  return launch_pdl(router_small_kernel, grid, dim3(128), smem, st, L, x, T, flags, logits, ids,
-                    w, ctl);
+  const size_t smem = router_small_smem(L.d, T);
+  cudaError_t e = cudaFuncSetAttribute(router_small_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((L.E + kRouterRows - 1) / kRouterRows);
+  return launch_pdl(router_small_kernel, grid, dim3(kRouterWarps * 32), smem, st, L, x, T, flags,
+                    logits, ids, w, ctl);
 }
 
 // ------------------------------------------------------------ prefill router
