@@ -83,16 +83,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete; gives up after
-// kWaitLimitNs, records kErrTimeout and returns false.
+// kWaitLimitNs, records kErrTimeout and returns false.  try_wait itself
+// suspends the thread for a while when the phase is not complete, so the loop
+// spins on it and reads the (slow) global timer only every 64 attempts.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Control* ctl,
                                           uint32_t where) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  for (;;) {
+  unsigned long long t0 = 0;
+  for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      record_error(ctl, kErrTimeout, where);
-      return false;
+    if ((n & 63u) == 0) {
+      const unsigned long long t = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = t;
+      } else if (t - t0 > kWaitLimitNs) {
+        record_error(ctl, kErrTimeout, where);
+        return false;
+      }
     }
   }
 }

@@ -143,6 +143,8 @@ WsLayout ws_layout(const LayerDev& L, int T) {
     o += align256(parts[7]);
     w.yacc = o;
     o += align256(parts[8]);
+    w.xperm = o;
+    o += align256(parts[9]);
   }
   w.total = o;
   return w;

@@ -23,12 +23,17 @@
 //  5. finalize y = bf16(y_acc (+ x)).
 //
 // Warp roles of the GEMM kernel (one CTA per SM, persistent over work items):
-//  warps 0-3  epilogue (TMEM lane quadrant = warp index)
-//  warps 4-7  A producers: packed codes arrive by bulk copy in a small ring;
-//             each thread dequantises one 128-byte row of the A tile
-//  warps 8-11 B producers: cp.async of token rows into the swizzled B tile
-//  warp 12    TMEM allocation and the single MMA-issuing thread
+//  warps 0-3   epilogue (TMEM lane quadrant = warp index)
+//  warps 4-11  A producers: each thread dequantises one 32-value group of a row
+//              of the A tile from the packed codes staged in a small ring
+//  warp 12     TMEM allocation and the single MMA-issuing thread
+//  warp 13     loads: the B tile of every k-step by TMA (rows of the permuted
+//              token buffer, or of H), and the packed codes by bulk copies
 // Every wait is bounded; a timed-out role records the error and stops waiting.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <string.h>
+
 #include "internal.h"
 #include "tc.cuh"
 
@@ -39,14 +44,20 @@ cudaError_t launch_prep_tokens(const uint16_t* x, int T, int d, uint32_t flags, 
 
 constexpr int PF_NT = 128;        // token tile = MMA N (max)
 constexpr int PF_BM = 128;        // MMA M
-constexpr int PF_NS = 4;          // operand ring stages
-constexpr int PF_CS = 4;          // packed-code ring stages
+constexpr int PF_NSA = 3;         // A (dequantised weights) ring stages: produced on chip
+constexpr int PF_NSB = 8;         // B (token rows) ring stages: loaded from memory by TMA
+constexpr int PF_CS = 8;          // packed-code ring stages
 constexpr int PF_TOKBLK = 256;    // bucketing token block
-constexpr int PF_CODE_SLOT = 448; // one 16-row tile in a code stage: lo 256 | hi 128 | scales 64
-constexpr int PF_CODE_STAGE = 8 * PF_CODE_SLOT;
+// Code stage of one k-step (two groups of 8 packed 16-row tiles), as the
+// 4-D tensor-map boxes land: [tile][group][bytes].
+//  gate/up: Wg lo [4][2][128] @0 | Wu lo @1024 | Wg hi [4][2][64] @2048 | Wu hi @2560
+//           | Wg scales [4][2][32] @3072 | Wu scales @3328
+//  down:    Wd lo [8][2][128] @0 | Wd hi [8][2][64] @2048 | Wd scales [8][2][32] @3072
+constexpr int PF_CODE_STAGE = 3584;
 constexpr int PF_A_STAGE = PF_BM * 128;
 constexpr int PF_B_STAGE = PF_NT * 128;
-constexpr int PF_THREADS = 13 * 32;
+constexpr int PF_THREADS = 14 * 32;
+constexpr int PF_A_THREADS = 256;
 
 struct PfWs {
   int* counts;      // [E+1]
@@ -61,6 +72,7 @@ struct PfWs {
   float* yacc;      // [T][d]
   __half* x16;      // [T][d]
   uint16_t* xn;     // [T][d]
+  __half* xperm;    // [T*(k+1)][d]: token rows in bucket order
 };
 
 static size_t pf_max_chunks(const LayerDev& L, int T) {
@@ -80,8 +92,9 @@ size_t prefill_ws_bytes(const LayerDev& L, int T, size_t* parts) {
   parts[6] = pf_max_chunks(L, T) * 16 + 256 + R * 4 + 256 + R * 4;   // chunks, tokpos, wpos
   parts[7] = (R + PF_NT) * Fmax * 2;                           // H
   parts[8] = (size_t)T * L.d * 4;                              // yacc
+  parts[9] = R * L.d * 2;                                      // xperm
   size_t tot = 0;
-  for (int i = 0; i < 9; ++i) tot += parts[i];
+  for (int i = 0; i < 10; ++i) tot += parts[i];
   return tot;
 }
 
@@ -103,6 +116,7 @@ static PfWs pf_ws(const LayerDev& L, int T, char* ws, const WsLayout& lay) {
   p.wpos = reinterpret_cast<float*>(t);
   p.H = reinterpret_cast<__half*>(ws + lay.h);
   p.yacc = reinterpret_cast<float*>(ws + lay.yacc);
+  p.xperm = reinterpret_cast<__half*>(ws + lay.xperm);
   return p;
 }
 
@@ -193,14 +207,14 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(int* __restrict__ blo
       p.chunks[nch[e] + c] = make_int4(e, off[e] + c * PF_NT, min(PF_NT, cnt[e] - c * PF_NT), 0);
   }
   if (tid == 0) {
-    p.offsets[E + 1] = off[E] + T;
+    p.offsets[E + 1] = off[E] + cnt[E];
     p.misc[0] = nchunks;
   }
 }
 
 __global__ void __launch_bounds__(256) bucket_scatter_kernel(const int32_t* __restrict__ ids,
                                                              const float* __restrict__ w, int T,
-                                                             int k, int E, PfWs p,
+                                                             int k, int E, int has_shared, PfWs p,
                                                              int32_t* __restrict__ user_entries) {
   extern __shared__ uint32_t bits[];   // [E][8]: token bitmap of this block per expert
   pdl_wait();
@@ -224,10 +238,36 @@ __global__ void __launch_bounds__(256) bucket_scatter_kernel(const int32_t* __re
     p.tokpos[pos] = t;
     p.wpos[pos] = w[i];
   }
-  for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
-    const int pos = T * k + t;
-    p.tokpos[pos] = t;
-    p.wpos[pos] = 1.f;
+  if (has_shared) {
+    for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
+      const int pos = p.offsets[E] + t;   // the shared bucket follows the routed ones
+      p.tokpos[pos] = t;
+      p.wpos[pos] = 1.f;
+    }
+  }
+}
+
+// Token rows in bucket order: xperm[pos] = x16[tokpos[pos]] for the filled
+// positions pos < offsets[E+1] (routed buckets, then the shared bucket).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __half* __restrict__ x16,
+                                                          const int* __restrict__ tokpos,
+                                                          const int* __restrict__ offsets, int E,
+                                                          int T, __half* __restrict__ xperm,
+                                                          int d, Control* ctl) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int per = d / 8;
+  const long long n = (long long)offsets[E + 1] * per;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long pos = i / per;
+    const int c = (int)(i - pos * per);
+    int t = tokpos[pos];
+    if (t < 0 || t >= T) {
+      record_error(ctl, kErrRange, 0x602);
+      t = 0;
+    }
+    reinterpret_cast<uint4*>(xperm)[i] = reinterpret_cast<const uint4*>(x16 + (size_t)t * d)[c];
   }
 }
 
@@ -245,7 +285,7 @@ struct PfArgs {
 };
 
 struct PfItem {
-  int u, pos0, nv, tile, F, K, KS;
+  int u, pos0, nv, tile, F, K, KS, slot;
   bool valid;
   const uint8_t* codes;
   const uint16_t* scales;
@@ -260,6 +300,7 @@ __device__ __forceinline__ PfItem pf_item(const PfArgs& a, int i, Control* ctl) 
   it.tile = i % a.tpc;
   if (it.u >= a.L.E) {
     it.F = a.L.Fs;
+    it.slot = 0;
     it.codes = a.L.scodes;
     it.scales = a.L.sscales;
   } else {
@@ -269,6 +310,7 @@ __device__ __forceinline__ PfItem pf_item(const PfArgs& a, int i, Control* ctl) 
       slot = 0;
     }
     it.F = a.L.F;
+    it.slot = slot;
     it.codes = a.L.codes + (long long)slot * a.L.cbe;
     it.scales = a.L.scales + (long long)slot * a.L.nse;
   }
@@ -314,58 +356,56 @@ struct KIter {
   }
 };
 
-// Packed-code tile slot q' (0..7) of an A tile: which packed 16-row tile feeds
-// it.  Returns false when the slot lies outside the matrix.
-__device__ __forceinline__ bool pf_slot(const PfArgs& a, const PfItem& it, int q, const uint8_t** mc,
-                                        const uint16_t** ms, int* tau, int* nGK) {
-  const int d = a.L.d;
-  const long long mcb = mat_codes_bytes(it.F, d, a.L.bits);
-  if (a.mode == 0) {
-    *tau = 4 * it.tile + (q >> 1);
-    *nGK = d / kGroup;
-    *mc = it.codes + ((q & 1) ? mcb : 0);
-    *ms = it.scales + ((q & 1) ? (long long)it.F * (d / kGroup) : 0);
-    return *tau < it.F / kTileRows;
-  }
-  *tau = 8 * it.tile + q;
-  *nGK = it.F / kGroup;
-  *mc = it.codes + 2 * mcb;
-  *ms = it.scales + 2LL * it.F * (d / kGroup);
-  return *tau < d / kTileRows;
+// Is packed tile slot q' (0..7) of the A tile inside the matrix?
+__device__ __forceinline__ bool pf_slot_valid(const PfArgs& a, const PfItem& it, int q) {
+  if (a.mode == 0) return 4 * it.tile + (q >> 1) < it.F / kTileRows;
+  return 8 * it.tile + q < a.L.d / kTileRows;
 }
 
-// warp-cooperative: bulk-copy the packed codes of k-step ks of `it` into a code stage
-__device__ __forceinline__ void pf_issue_codes(const PfArgs& a, const PfItem& it, int ks,
-                                               unsigned char* stage, uint64_t* bar) {
-  const int lane = threadIdx.x & 31;
-  const int bits = a.L.bits;
-  const int gbase = 2 * ks;
-  const int ng = min(2, it.K / kGroup - gbase);
-  uint32_t total = 0;
-  for (int q = 0; q < 8; ++q) {
-    const uint8_t* mc;
-    const uint16_t* ms;
-    int tau, nGK;
-    if (pf_slot(a, it, q, &mc, &ms, &tau, &nGK)) total += ng * (128 + 32 + (bits == 3 ? 64 : 0));
-  }
-  if (lane == 0) mbar_arrive_expect_tx(bar, total);
-  __syncwarp();
-  if (lane < 24) {
-    const int q = lane / 3, part = lane % 3;
-    const uint8_t* mc;
-    const uint16_t* ms;
-    int tau, nGK;
-    if (pf_slot(a, it, q, &mc, &ms, &tau, &nGK)) {
-      const long long tcb = (long long)nGK * kTileRows * group_bytes(bits);
-      unsigned char* dst = stage + q * PF_CODE_SLOT;
-      if (part == 0) {
-        bulk_g2s(dst, mc + tau * tcb + gbase * 128, ng * 128, bar);
-      } else if (part == 1) {
-        if (bits == 3) bulk_g2s(dst + 256, mc + tau * tcb + nGK * 128 + gbase * 64, ng * 64, bar);
-      } else {
-        bulk_g2s(dst + 384, ms + (long long)tau * kTileRows * nGK + gbase * 16, ng * 32, bar);
-      }
+// Tensor maps: the token (or hidden) rows of the B operand, and the packed
+// codes / scales of the routed experts and of the shared expert viewed as
+// 4-D byte tensors [bytes of a group][group][16-row tile][slot].
+struct alignas(64) PfMaps {
+  CUtensorMap b;
+  CUtensorMap lo, hi, sc;      // routed experts
+  CUtensorMap slo, shi, ssc;   // shared expert
+};
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+// One lane: the packed codes and scales of k-step ks of `it` into a code stage.
+__device__ __forceinline__ void pf_issue_codes(const PfArgs& a, const PfMaps& mp, const PfItem& it,
+                                               int ks, unsigned char* st, uint64_t* bar) {
+  const bool sh = it.u >= a.L.E;
+  const CUtensorMap* lo = sh ? &mp.slo : &mp.lo;
+  const CUtensorMap* hi = sh ? &mp.shi : &mp.hi;
+  const CUtensorMap* sc = sh ? &mp.ssc : &mp.sc;
+  const int g0 = 2 * ks, bits = a.L.bits;
+  if (a.mode == 0) {
+    const int t0 = 4 * it.tile, tu = it.F / kTileRows + 4 * it.tile;
+    mbar_arrive_expect_tx(bar, 2 * (1024 + 256) + (bits == 3 ? 1024 : 0));
+    tma_load_4d(st, lo, 0, g0, t0, it.slot, bar);
+    tma_load_4d(st + 1024, lo, 0, g0, tu, it.slot, bar);
+    if (bits == 3) {
+      tma_load_4d(st + 2048, hi, 0, g0, t0, it.slot, bar);
+      tma_load_4d(st + 2560, hi, 0, g0, tu, it.slot, bar);
     }
+    tma_load_4d(st + 3072, sc, 0, g0, t0, it.slot, bar);
+    tma_load_4d(st + 3328, sc, 0, g0, tu, it.slot, bar);
+  } else {
+    const int t0 = 8 * it.tile;
+    mbar_arrive_expect_tx(bar, 2048 + 512 + (bits == 3 ? 1024 : 0));
+    tma_load_4d(st, lo, 0, g0, t0, it.slot, bar);
+    if (bits == 3) tma_load_4d(st + 2048, hi, 0, g0, t0, it.slot, bar);
+    tma_load_4d(st + 3072, sc, 0, g0, t0, it.slot, bar);
   }
 }
 
@@ -397,27 +437,39 @@ __device__ __forceinline__ uint4 pf_dq_chunk(const uint32_t (&X)[4], const uint3
 }
 
 struct PfSmem {
-  size_t a, b, codes, bars, holder, total;
+  size_t a, b, codes, stage_h, bars, holder, total;
 };
 __host__ __device__ inline PfSmem pf_smem() {
   PfSmem m;
   size_t o = 0;
   m.a = o;
-  o += (size_t)PF_NS * PF_A_STAGE;
+  o += (size_t)PF_NSA * PF_A_STAGE;
   m.b = o;
-  o += (size_t)PF_NS * PF_B_STAGE;
+  o += (size_t)PF_NSB * PF_B_STAGE;
   m.codes = o;
   o += (size_t)PF_CS * PF_CODE_STAGE;
+  m.stage_h = o;                       // epilogue staging of H rows: [128 n][64 f] fp16
+  o += (size_t)PF_NT * 64 * 2;
   m.bars = o;
-  o += (2 * PF_NS + PF_CS + 4) * 8;
+  o += (2 * PF_NSA + 2 * PF_NSB + 2 * PF_CS + 4) * 8;
   m.holder = o;
   o += 16;
   m.total = o + 1024;   // slack to align the base to 1024
   return m;
 }
 
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
 template <int BITS>
-__global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a) {
+__global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
+                                                                 const __grid_constant__ PfMaps mp) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -425,21 +477,32 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a) 
   unsigned char* sA = smem + m.a;
   unsigned char* sB = smem + m.b;
   unsigned char* sC = smem + m.codes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + m.bars);
-  uint64_t* empty = full + PF_NS;
-  uint64_t* cfull = empty + PF_NS;
-  uint64_t* tfull = cfull + PF_CS;
+  __half* sH = reinterpret_cast<__half*>(smem + m.stage_h);
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + m.bars);
+  uint64_t* emptyA = fullA + PF_NSA;
+  uint64_t* fullB = emptyA + PF_NSA;
+  uint64_t* emptyB = fullB + PF_NSB;
+  uint64_t* cfull = emptyB + PF_NSB;
+  uint64_t* cempty = cfull + PF_CS;
+  uint64_t* tfull = cempty + PF_CS;
   uint64_t* tempty = tfull + 2;
   uint32_t* holder = reinterpret_cast<uint32_t*>(smem + m.holder);
   Control* ctl = a.ctl;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    for (int s = 0; s < PF_NS; ++s) {
-      mbar_init(&full[s], 256);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < PF_NSA; ++s) {
+      mbar_init(&fullA[s], PF_A_THREADS);
+      mbar_init(&emptyA[s], 1);
     }
-    for (int c = 0; c < PF_CS; ++c) mbar_init(&cfull[c], 1);
+    for (int s = 0; s < PF_NSB; ++s) {
+      mbar_init(&fullB[s], 1);
+      mbar_init(&emptyB[s], 1);
+    }
+    for (int c = 0; c < PF_CS; ++c) {
+      mbar_init(&cfull[c], 1);
+      mbar_init(&cempty[c], PF_A_THREADS);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 128);
@@ -450,6 +513,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a) 
     tmem_alloc(holder, 512);
     tmem_relinquish();
   }
+  if (warp == 13 && lane < 7) {   // the seven tensor-map descriptors into the TMA unit's cache
+    const CUtensorMap* maps[7] = {&mp.b, &mp.lo, &mp.hi, &mp.sc, &mp.slo, &mp.shi, &mp.ssc};
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(maps[lane])) : "memory");
+  }
   pdl_wait();
   pdl_launch_dependents();
   tc_fence_before();
@@ -459,16 +526,24 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a) 
   const int n_items = a.p.misc[0] * a.tpc;
   bool ok = true;
 
-  if (warp >= 4 && warp < 8) {
+  if (warp >= 4 && warp < 12) {
     // ------------------------------------------------ A producers (dequant)
-    const int r = tid - 128;
-    KIter ahead;   // issuer's iterator, PF_CS k-steps ahead
-    if (warp == 4) {
-      ahead.init(a, n_items, ctl);
-      for (int c = 0; c < PF_CS && !ahead.done; ++c) {
-        pf_issue_codes(a, ahead.item, ahead.ks, sC + c * PF_CODE_STAGE, &cfull[c]);
-        ahead.advance(a, ctl);
-      }
+    const int ta = tid - 128;
+    const int r = ta >> 1, gi = ta & 1;
+    int q, rr, lo_off, hi_off, sc_off;
+    if (a.mode == 0) {
+      const int qt = r >> 5, isu = ((r & 31) >> 4) & 1;
+      q = 2 * qt + isu;
+      rr = r & 15;
+      lo_off = isu * 1024 + qt * 256;
+      hi_off = 2048 + isu * 512 + qt * 128;
+      sc_off = 3072 + isu * 256 + qt * 64;
+    } else {
+      q = r >> 4;
+      rr = r & 15;
+      lo_off = q * 256;
+      hi_off = 2048 + q * 128;
+      sc_off = 3072 + q * 64;
     }
     KIter cur;
     cur.init(a, n_items, ctl);
@@ -477,109 +552,69 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a) 
       const PfItem& it = cur.item;
       const int cs = g % PF_CS;
       if (ok) ok = mbar_wait(&cfull[cs], (g / PF_CS) & 1, ctl, 0x610);
-      const unsigned char* cst = sC + cs * PF_CODE_STAGE;
-      int q, rr;
-      if (a.mode == 0) {
-        q = 2 * (r >> 5) + (((r & 31) >> 4) & 1);
-        rr = r & 15;
-      } else {
-        q = r >> 4;
-        rr = r & 15;
-      }
-      const uint8_t* mc;
-      const uint16_t* ms;
-      int tau, nGK;
-      const bool rv = pf_slot(a, it, q, &mc, &ms, &tau, &nGK);
+      const bool rv = pf_slot_valid(a, it, q);
       const int ng = min(2, it.K / kGroup - 2 * cur.ks);
-      uint4 chunk[8];
+      const bool mine = rv && gi < ng && ok;
+      uint32_t X[4], Y[4];
+      __half2 s2 = __float2half2_rn(0.f);
+      if (mine) {
+        const unsigned char* cst = sC + cs * PF_CODE_STAGE;
+        const uint2 lo = *reinterpret_cast<const uint2*>(cst + lo_off + gi * 128 + rr * 8);
+        const uint32_t hi = BITS == 3 ? *reinterpret_cast<const uint32_t*>(cst + hi_off + gi * 64 + rr * 4) : 0u;
+        s2 = __half2half2(*reinterpret_cast<const __half*>(cst + sc_off + gi * 32 + rr * 2));
 #pragma unroll
-      for (int gi = 0; gi < 2; ++gi) {
-        uint32_t X[4], Y[4];
-        __half2 s2 = __float2half2_rn(0.f);
-        if (rv && gi < ng && ok) {
-          const unsigned char* slot = cst + q * PF_CODE_SLOT;
-          const uint2 lo = *reinterpret_cast<const uint2*>(slot + (gi * 16 + rr) * 8);
-          const uint32_t hi = BITS == 3 ? *reinterpret_cast<const uint32_t*>(slot + 256 + (gi * 16 + rr) * 4) : 0u;
-          const __half s = *reinterpret_cast<const __half*>(slot + 384 + (gi * 16 + rr) * 2);
-          s2 = __half2half2(s);
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            X[t] = __byte_perm(lo.x, lo.y, (uint32_t)t | ((uint32_t)(4 + t) << 8));
-            Y[t] = hi >> (4 * t);
-          }
-        } else {
-#pragma unroll
-          for (int t = 0; t < 4; ++t) X[t] = Y[t] = 0u;
+        for (int t = 0; t < 4; ++t) {
+          X[t] = __byte_perm(lo.x, lo.y, (uint32_t)t | ((uint32_t)(4 + t) << 8));
+          Y[t] = hi >> (4 * t);
         }
+      } else {
 #pragma unroll
-        for (int mm = 0; mm < 4; ++mm) chunk[gi * 4 + mm] = pf_dq_chunk<BITS>(X, Y, mm, s2);
+        for (int t = 0; t < 4; ++t) X[t] = Y[t] = 0u;
       }
-      named_bar_sync(2, 128);   // every A thread has read code stage cs
-      if (warp == 4 && !ahead.done) {
-        pf_issue_codes(a, ahead.item, ahead.ks, sC + cs * PF_CODE_STAGE, &cfull[cs]);
-        ahead.advance(a, ctl);
-      }
-      const int s = g % PF_NS;
-      if (g >= PF_NS && ok) ok = mbar_wait(&empty[s], ((g / PF_NS) - 1) & 1, ctl, 0x611);
-      unsigned char* at = sA + s * PF_A_STAGE + r * 128;
+      mbar_arrive(&cempty[cs]);   // code stage read
+      uint4 chunk[4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(at + ((c ^ (r & 7)) << 4)) = chunk[c];
+      for (int mm = 0; mm < 4; ++mm) chunk[mm] = pf_dq_chunk<BITS>(X, Y, mm, s2);
+      const int s = g % PF_NSA;
+      if (g >= PF_NSA && ok) ok = mbar_wait(&emptyA[s], ((g / PF_NSA) - 1) & 1, ctl, 0x611);
+      if (gi < ng) {
+        unsigned char* at = sA + s * PF_A_STAGE + r * 128;
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+          const int c = 4 * gi + mm;
+          *reinterpret_cast<uint4*>(at + ((c ^ (r & 7)) << 4)) = chunk[mm];
+        }
+      }
       fence_proxy_async_smem();
-      mbar_arrive(&full[s]);
+      mbar_arrive(&fullA[s]);
       cur.advance(a, ctl);
       ++g;
     }
-  } else if (warp >= 8 && warp < 12) {
-    // ------------------------------------------------ B producers (rows)
-    const int b = tid - 256;
-    const int c = b & 7;
-    KIter cur;
+  } else if (warp == 13) {
+    // ------------------------------------------------ loads (TMA / bulk)
+    KIter cur, ahead;
     cur.init(a, n_items, ctl);
-    int g = 0, prev_s = -1;
-    const __half* rows[8];
-    int cur_it = -1;
+    ahead.init(a, n_items, ctl);
+    int g = 0, gc = 0;
     while (!cur.done) {
-      const PfItem& it = cur.item;
-      const int n_mma = (it.nv + 15) & ~15;
-      if (cur.it != cur_it) {
-        cur_it = cur.it;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int n = (b >> 3) + 16 * i;
-          rows[i] = a.bsrc;
-          if (n < it.nv) {
-            const int row = a.mode == 0 ? a.p.tokpos[it.pos0 + n] : it.pos0 + n;
-            rows[i] = a.bsrc + (size_t)row * a.bstride;
-          }
-        }
+      // packed codes up to PF_CS k-steps ahead of the B loads
+      while (!ahead.done && gc < g + PF_CS) {
+        const int cs = gc % PF_CS;
+        if (gc >= PF_CS && ok) ok = mbar_wait(&cempty[cs], ((gc / PF_CS) - 1) & 1, ctl, 0x621);
+        if (lane == 0) pf_issue_codes(a, mp, ahead.item, ahead.ks, sC + cs * PF_CODE_STAGE, &cfull[cs]);
+        ahead.advance(a, ctl);
+        ++gc;
       }
-      const int s = g % PF_NS;
-      if (g >= PF_NS && ok) ok = mbar_wait(&empty[s], ((g / PF_NS) - 1) & 1, ctl, 0x620);
-      const int nc = 4 * min(2, it.K / kGroup - 2 * cur.ks);
-      unsigned char* bt = sB + s * PF_B_STAGE;
-      if (c < nc && ok) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int n = (b >> 3) + 16 * i;
-          if (n < n_mma)
-            cp_async16(bt + n * 128 + ((c ^ (n & 7)) << 4), rows[i] + 64 * cur.ks + 8 * c,
-                       n < it.nv ? 16u : 0u);
-        }
+      const int s = g % PF_NSB;
+      if (g >= PF_NSB && ok) ok = mbar_wait(&emptyB[s], ((g / PF_NSB) - 1) & 1, ctl, 0x620);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&fullB[s], PF_B_STAGE);
+        tma_load_2d(sB + s * PF_B_STAGE, &mp.b, 64 * cur.ks, cur.item.pos0, &fullB[s]);
       }
-      cp_async_commit();
-      if (prev_s >= 0) {
-        cp_async_wait<1>();
-        fence_proxy_async_smem();
-        mbar_arrive(&full[prev_s]);
-      }
-      prev_s = s;
+      __syncwarp();
       cur.advance(a, ctl);
       ++g;
     }
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    if (prev_s >= 0) mbar_arrive(&full[prev_s]);
   } else if (warp == 12) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -595,18 +630,20 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a) 
         const uint32_t idesc = idesc_f16_f32(PF_BM, n_mma);
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
         for (int ks = 0; ks < it.KS; ++ks) {
-          const int s = g % PF_NS;
-          if (ok) ok = mbar_wait(&full[s], (g / PF_NS) & 1, ctl, 0x631);
+          const int sa = g % PF_NSA, sb = g % PF_NSB;
+          if (ok) ok = mbar_wait(&fullB[sb], (g / PF_NSB) & 1, ctl, 0x632);
+          if (ok) ok = mbar_wait(&fullA[sa], (g / PF_NSA) & 1, ctl, 0x631);
           tc_fence_after();
           const int nk = 2 * min(2, it.K / kGroup - 2 * ks);
-          const uint32_t abase = smem_u32(sA + s * PF_A_STAGE);
-          const uint32_t bbase = smem_u32(sB + s * PF_B_STAGE);
+          const uint32_t abase = smem_u32(sA + sa * PF_A_STAGE);
+          const uint32_t bbase = smem_u32(sB + sb * PF_B_STAGE);
           if (ok) {
             for (int kk = 0; kk < nk; ++kk)
               tc_mma_f16(d_tmem, sw128_kmajor_desc(abase + kk * 32), sw128_kmajor_desc(bbase + kk * 32),
                          idesc, (ks | kk) != 0);
           }
-          tc_commit(&empty[s]);
+          tc_commit(&emptyA[sa]);
+          tc_commit(&emptyB[sb]);
           ++g;
         }
         tc_commit(&tfull[acc]);
@@ -628,8 +665,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a) 
       const int n_mma = (it.nv + 15) & ~15;
       const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * 256);
       if (a.mode == 0) {
-        const int f = 64 * it.tile + 16 * q + (lane & 15);
-        const bool wr = lane < 16 && f < it.F;
+        // SwiGLU into the staging tile sH[n][64 f], then coalesced row stores
+        const int fl = 16 * q + (lane & 15);
         for (int c0 = 0; c0 < n_mma; c0 += 32) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(taddr + c0, v);
@@ -638,13 +675,20 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a) 
           for (int j = 0; j < 32; ++j) {
             const float gv = __uint_as_float(v[j]);
             const float up = __shfl_xor_sync(0xffffffffu, gv, 16);
-            const int n = c0 + j;
-            if (wr && n < it.nv && ok) {
-              const float h = gv / (1.f + expf(-gv)) * up;
-              a.p.H[(size_t)(it.pos0 + n) * a.Fmax + f] = __float2half_rn(h);
-            }
+            if (lane < 16) sH[(c0 + j) * 64 + fl] = __float2half_rn(gv / (1.f + expf(-gv)) * up);
           }
         }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);   // TMEM free: the MMA may start the next item
+        named_bar_sync(3, 128);
+        const int fcol = 64 * it.tile + 2 * lane;
+        if (ok && fcol < it.F) {
+          for (int n = q; n < it.nv; n += 4) {
+            const uint32_t hv = *reinterpret_cast<const uint32_t*>(sH + n * 64 + 2 * lane);
+            *reinterpret_cast<uint32_t*>(a.p.H + (size_t)(it.pos0 + n) * a.Fmax + fcol) = hv;
+          }
+        }
+        named_bar_sync(3, 128);
       } else {
         const int i_out = PF_BM * it.tile + 32 * q + lane;
         const bool wr = i_out < a.L.d;
@@ -662,9 +706,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a) 
             }
           }
         }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
       ++la;
       cur.next_item(a, ctl);
     }
@@ -699,13 +743,77 @@ __global__ void __launch_bounds__(256) prefill_finalize_kernel(const float* __re
   }
 }
 
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D fp16 row-major tensor [rows][inner] for tiles of PF_NT rows x 64
+// elements, 128-byte swizzle (the canonical K-major UMMA layout).
+static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, PF_NT};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 4-D byte tensor [inner bytes][groups][tiles][slots] with the given strides.
+static bool make_map4(CUtensorMap* m, const void* base, uint64_t inner, uint64_t groups,
+                      uint64_t tiles, uint64_t slots, uint64_t s_group, uint64_t s_tile,
+                      uint64_t s_slot, uint32_t box_tiles) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {inner, groups, tiles, slots};
+  cuuint64_t strides[3] = {s_group, s_tile, s_slot};
+  cuuint32_t box[4] = {(cuuint32_t)inner, 2, box_tiles, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Maps of one expert set (routed: E slots, or the shared expert: 1 slot).
+static bool make_code_maps(const LayerDev& L, int mode, const uint8_t* codes, const uint16_t* scales,
+                           int F, uint64_t slots, CUtensorMap* lo, CUtensorMap* hi, CUtensorMap* sc) {
+  const int gb = group_bytes(L.bits);
+  const uint64_t cbe = 3ull * F * L.d / kGroup * gb, nse2 = 3ull * F * L.d / kGroup * 2;
+  const uint64_t nG = L.d / kGroup, nGF = F / kGroup;
+  const uint64_t tcb = nG * kTileRows * gb, tcbD = nGF * kTileRows * gb;
+  const uint64_t mcb = (uint64_t)(F / kTileRows) * tcb;
+  const uint64_t sslot = cbe, sslot_s = nse2;   // slot strides (unused when slots == 1)
+  if (mode == 0) {
+    const uint64_t tiles = 2ull * F / kTileRows;
+    return make_map4(lo, codes, 128, nG, tiles, slots, 128, tcb, sslot, 4) &&
+           (L.bits == 2 || make_map4(hi, codes + nG * 128, 64, nG, tiles, slots, 64, tcb, sslot, 4)) &&
+           make_map4(sc, scales, 32, nG, tiles, slots, 32, 32 * nG, sslot_s, 4);
+  }
+  const uint64_t tiles = (uint64_t)L.d / kTileRows;
+  const uint8_t* wd = codes + 2 * mcb;
+  const uint8_t* wds = reinterpret_cast<const uint8_t*>(scales) + 2ull * F * nG * 2;
+  return make_map4(lo, wd, 128, nGF, tiles, slots, 128, tcbD, sslot, 8) &&
+         (L.bits == 2 || make_map4(hi, wd + nGF * 128, 64, nGF, tiles, slots, 64, tcbD, sslot, 8)) &&
+         make_map4(sc, wds, 32, nGF, tiles, slots, 32, 32 * nGF, sslot_s, 8);
+}
+
 template <int BITS>
-static cudaError_t launch_gemm(const PfArgs& a, cudaStream_t st) {
+static cudaError_t launch_gemm(const PfArgs& a, const PfMaps& tm, cudaStream_t st) {
   const PfSmem m = pf_smem();
   cudaError_t e = cudaFuncSetAttribute(pf_gemm_kernel<BITS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)m.total);
   if (e != cudaSuccess) return e;
-  return launch_pdl(pf_gemm_kernel<BITS>, dim3(sm_count()), dim3(PF_THREADS), m.total, st, a);
+  return launch_pdl(pf_gemm_kernel<BITS>, dim3(sm_count()), dim3(PF_THREADS), m.total, st, a, tm);
 }
 
 cudaError_t launch_prefill(const LayerDev& L, const uint16_t* x, int T, const int32_t* ids,
@@ -726,8 +834,24 @@ cudaError_t launch_prefill(const LayerDev& L, const uint16_t* x, int T, const in
                  L.Fs > 0 ? 1 : 0, p, offsets_out);
   if (e != cudaSuccess) return e;
   e = launch_pdl(bucket_scatter_kernel, dim3(nblk), dim3(256), (size_t)L.E * 32, st, ids, w, T, L.k,
-                 L.E, p, entries_out);
+                 L.E, L.Fs > 0 ? 1 : 0, p, entries_out);
   if (e != cudaSuccess) return e;
+  const size_t R = (size_t)T * (L.k + 1);
+  e = launch_pdl(gather_rows_kernel, dim3(4 * sm_count()), dim3(256), 0, st,
+                 static_cast<const __half*>(p.x16), static_cast<const int*>(p.tokpos),
+                 static_cast<const int*>(p.offsets), L.E, T, p.xperm, L.d, ctl);
+  if (e != cudaSuccess) return e;
+  PfMaps m0, m1;
+  memset(&m0, 0, sizeof m0);
+  memset(&m1, 0, sizeof m1);
+  if (!make_map(&m0.b, p.xperm, (uint64_t)L.d, (uint64_t)R) ||
+      !make_map(&m1.b, p.H, (uint64_t)Fmax, (uint64_t)(R + PF_NT)) ||
+      !make_code_maps(L, 0, L.codes, L.scales, L.F, L.E, &m0.lo, &m0.hi, &m0.sc) ||
+      !make_code_maps(L, 1, L.codes, L.scales, L.F, L.E, &m1.lo, &m1.hi, &m1.sc))
+    return cudaErrorInvalidValue;
+  if (L.Fs > 0 && (!make_code_maps(L, 0, L.scodes, L.sscales, L.Fs, 1, &m0.slo, &m0.shi, &m0.ssc) ||
+                   !make_code_maps(L, 1, L.scodes, L.sscales, L.Fs, 1, &m1.slo, &m1.shi, &m1.ssc)))
+    return cudaErrorInvalidValue;
   PfArgs a;
   a.L = L;
   a.T = T;
@@ -735,16 +859,16 @@ cudaError_t launch_prefill(const LayerDev& L, const uint16_t* x, int T, const in
   a.p = p;
   a.mode = 0;
   a.tpc = (Fmax + 63) / 64;
-  a.bsrc = p.x16;
+  a.bsrc = p.xperm;
   a.bstride = L.d;
   a.ctl = ctl;
-  e = L.bits == 2 ? launch_gemm<2>(a, st) : launch_gemm<3>(a, st);
+  e = L.bits == 2 ? launch_gemm<2>(a, m0, st) : launch_gemm<3>(a, m0, st);
   if (e != cudaSuccess) return e;
   a.mode = 1;
   a.tpc = (L.d + PF_BM - 1) / PF_BM;
   a.bsrc = p.H;
   a.bstride = Fmax;
-  e = L.bits == 2 ? launch_gemm<2>(a, st) : launch_gemm<3>(a, st);
+  e = L.bits == 2 ? launch_gemm<2>(a, m1, st) : launch_gemm<3>(a, m1, st);
   if (e != cudaSuccess) return e;
   const long long n4 = (long long)T * L.d / 4;
   int grid = (int)((n4 + 255) / 256);

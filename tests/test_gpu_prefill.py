@@ -103,3 +103,24 @@ def test_prefill_full_size_chunk():
     print("experts hit", int((counts > 0).sum()), "median", int(np.median(counts)),
           "max", int(counts.max()))
     assert gb.error_word() == (0, 0)
+
+
+def test_prefill_out_of_range_ids_are_flagged_not_read():
+    sh = synth.MoEShape(d=128, E=32, F=64, Fs=64, k=4, bits=2)
+    layer = synth.make_layer(sh, seed=1, device="cuda", bias="normal")
+    T = 40
+    x = synth.make_tokens(T, 128, seed=2, device="cuda")
+    gb = GpuBlock(layer, T)
+    _, ids, w = gb.route(x)
+    bad = ids.clone()
+    bad[3, 1] = 99
+    bad[17, 0] = -5
+    y = gb.prefill(x, bad, w)
+    torch.cuda.synchronize()
+    st, code = gb.error_word()
+    assert st == 6 and code & 2
+    assert torch.isfinite(y.float()).all()
+    # tokens untouched by the bad entries match the clean run
+    y_ok = gb.prefill(x, ids, w)
+    keep = [t for t in range(T) if t not in (3, 17)]
+    assert torch.equal(y[keep], y_ok[keep])
