@@ -45,7 +45,7 @@ struct WsLayout {
   size_t tiles;      // prefill: int32 work list
   size_t h;          // prefill: fp16 hidden [rows][Fmax]
   size_t yacc;       // prefill: fp32 [T][d]
-  size_t xperm;      // prefill: fp16 [T*(k+1)][d]
+  size_t xperm;      // prefill: fp16 xperm / fp32 ybuf [T*(k+1)][d]
   size_t total;
 };
 WsLayout ws_layout(const LayerDev& L, int T);

@@ -124,3 +124,61 @@ def test_prefill_out_of_range_ids_are_flagged_not_read():
     y_ok = gb.prefill(x, ids, w)
     keep = [t for t in range(T) if t not in (3, 17)]
     assert torch.equal(y[keep], y_ok[keep])
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_prefill_deterministic_mode(bits):
+    """MOE_F_DETERMINISTIC: the fixed-order combine matches the oracle, repeats
+    bit for bit, and agrees with the reducing combine within rounding."""
+    sh = synth.MoEShape(d=256, E=48, F=128, Fs=96, k=6, bits=bits)
+    layer = synth.make_layer(sh, seed=9, device="cuda", bias="normal", bias_std=1.0)
+    T = 900
+    x = synth.make_tokens(T, sh.d, seed=5, device="cuda")
+    gb = GpuBlock(layer, T)
+    logits, ids, w = gb.route(x)
+    f = moe.F_DETERMINISTIC | moe.F_RESIDUAL
+    y1 = gb.prefill(x, ids, w, f)
+    y2 = gb.prefill(x, ids, w, f)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    oracle_check(layer, x, logits, ids, w, y1, flags=moe.F_RESIDUAL)
+    y3 = gb.prefill(x, ids, w, moe.F_RESIDUAL)
+    assert_close(y3.float().cpu().double().numpy(), y1.float().cpu().double().numpy(),
+                 max_rel=1e-2, rms_rel=1e-3)
+    assert gb.error_word() == (0, 0)
+
+
+def test_prefill_deterministic_slot_layout_invariance():
+    """The same experts packed into other slots: bit-identical deterministic
+    prefill output."""
+    sh = synth.MoEShape(d=256, E=64, F=128, Fs=128, k=6, bits=3)
+    a = synth.make_layer(sh, seed=4, device="cuda", bias="normal", slot="identity")
+    b = synth.make_layer(sh, seed=4, device="cuda", bias="normal", slot="random")
+    assert not torch.equal(a.expert_slot, b.expert_slot)
+    T = 500
+    x = synth.make_tokens(T, 256, seed=8, device="cuda")
+    ga, gb = GpuBlock(a, T), GpuBlock(b, T)
+    _, ids, w = ga.route(x)
+    ya = ga.prefill(x, ids, w, moe.F_DETERMINISTIC)
+    yb = gb.prefill(x, ids, w, moe.F_DETERMINISTIC)
+    torch.cuda.synchronize()
+    assert torch.equal(ya, yb)
+
+
+def test_prefill_full_size_deterministic_matches_sampled_oracle():
+    """8192-token chunk with the fixed-order combine: sampled rows against the
+    oracle and bitwise repeatability."""
+    wl = synth.WORKLOADS["prefill"]
+    layer = synth.make_layer(wl["shape"], seed=1, device="cuda", bias=wl["bias"],
+                             bias_std=wl["bias_std"], slot=wl["slot"])
+    T = wl["T"]
+    x = synth.make_tokens(T, 2048, seed=1, device="cuda")
+    gb = GpuBlock(layer, T)
+    logits, ids, w = gb.route(x)
+    y1 = gb.prefill(x, ids, w, moe.F_DETERMINISTIC)
+    y2 = gb.prefill(x, ids, w, moe.F_DETERMINISTIC)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    rows = np.random.default_rng(1).choice(T, 48, replace=False)
+    oracle_check(layer, x, logits, ids, w, y1, rows=rows)
+    assert gb.error_word() == (0, 0)
