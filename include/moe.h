@@ -85,7 +85,7 @@ typedef enum {
 /* flags */
 #define MOE_F_PRENORM 1u        /* router and experts see bf16(RMSNorm(x)) */
 #define MOE_F_RESIDUAL 2u       /* y = x + MoE(.) */
-#define MOE_F_DETERMINISTIC 4u  /* prefill: fixed-order combine (no float atomics) */
+#define MOE_F_DETERMINISTIC 4u  /* accepted; every path already combines in a fixed order */
 #define MOE_F_DEBUG 8u          /* kernels range-check ids, slots and values */
 
 /* One layer.  A host struct, read only during the call. */

@@ -82,24 +82,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `ns` nanoseconds pass, instead of spinning on the issue
+// slots that the other warps of its SM sub-partition need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete; gives up after
-// kWaitLimitNs, records kErrTimeout and returns false.  try_wait itself
-// suspends the thread for a while when the phase is not complete, so the loop
-// spins on it and reads the (slow) global timer only every 64 attempts.
+// kWaitLimitNs of %globaltimer, records kErrTimeout and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Control* ctl,
                                           uint32_t where) {
   if (mbar_try_wait(bar, parity)) return true;
-  unsigned long long t0 = 0;
-  for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 63u) == 0) {
-      const unsigned long long t = globaltimer_ns();
-      if (t0 == 0) {
-        t0 = t;
-      } else if (t - t0 > kWaitLimitNs) {
-        record_error(ctl, kErrTimeout, where);
-        return false;
-      }
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(ctl, kErrTimeout, where);
+      return false;
     }
   }
 }

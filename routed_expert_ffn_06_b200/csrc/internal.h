@@ -44,8 +44,9 @@ struct WsLayout {
   size_t blockcnt;   // prefill: int32 [nblk][E]
   size_t tiles;      // prefill: int32 work list
   size_t h;          // prefill: fp16 hidden [rows][Fmax]
-  size_t yacc;       // prefill: fp32 [T][d]
-  size_t xperm;      // prefill: fp16 xperm / fp32 ybuf [T*(k+1)][d]
+  size_t yacc;       // (unused, zero bytes)
+  size_t xperm;      // prefill: fp16 [T*(k+1)][d]: xperm (GEMM1 operand), then ybuf (GEMM2 output)
+  size_t wsplit;     // T > decode window: router weights as bf16 hi and lo [2][E][d]
   size_t total;
 };
 WsLayout ws_layout(const LayerDev& L, int T);
@@ -55,8 +56,10 @@ cudaError_t launch_router_small(const LayerDev& L, const uint16_t* x, int T, uin
                                 float* logits, int32_t* ids, float* w, Control* ctl,
                                 cudaStream_t st);
 cudaError_t launch_router_large(const LayerDev& L, const uint16_t* x, int T, uint32_t flags,
-                                float* logits, int32_t* ids, float* w, Control* ctl,
-                                cudaStream_t st);
+                                float* logits, int32_t* ids, float* w, uint16_t* wsplit,
+                                Control* ctl, cudaStream_t st);
+cudaError_t launch_router_tc(const LayerDev& L, const uint16_t* x, int T, float* logits,
+                             uint16_t* hi, uint16_t* lo, Control* ctl, cudaStream_t st);
 cudaError_t launch_decode(const LayerDev& L, const uint16_t* x, int T, const int32_t* ids,
                           const float* w, uint16_t* y, uint32_t flags, char* ws, const WsLayout& lay,
                           cudaStream_t st);

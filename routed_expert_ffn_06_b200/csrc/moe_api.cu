@@ -146,6 +146,10 @@ WsLayout ws_layout(const LayerDev& L, int T) {
     w.xperm = o;
     o += align256(parts[9]);
   }
+  if (T > kMaxDecodeT) {
+    w.wsplit = o;
+    o += align256((size_t)2 * L.E * L.d * sizeof(uint16_t));
+  }
   w.total = o;
   return w;
 }
@@ -210,7 +214,8 @@ moe_status moe_route_topk(const moe_layer* layer, const void* x_bf16, int32_t T,
     if (e != cudaSuccess) return from_cuda(e);
     xr = reinterpret_cast<const uint16_t*>(w + lay.xn);
   }
-  return from_cuda(launch_router_large(L, xr, T, flags, logits, topk_ids, topk_w, ctl, st));
+  return from_cuda(launch_router_large(L, xr, T, flags, logits, topk_ids, topk_w,
+                                       reinterpret_cast<uint16_t*>(w + lay.wsplit), ctl, st));
 }
 
 moe_status moe_expert_ffn_decode(const moe_layer* layer, const void* x_bf16, int32_t T,

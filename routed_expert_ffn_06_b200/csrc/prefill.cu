@@ -21,18 +21,23 @@
 //              (fp16).
 //  5. GEMM2:   for each (chunk, pair of 128-row tiles of d): D = Wd_tile .
 //              H_chunk^T; the epilogue scales column n by its routing weight
-//              and adds it into y_acc[token][i] (fp32 reductions), or, with
-//              MOE_F_DETERMINISTIC, stores it as row `position` of ybuf.
-//  6. finalize y = bf16(y_acc (+ x)), or the fixed-order sum of the ybuf rows
-//              of each token (+ x).
+//              and stores it as row `position` of ybuf (fp16, plain coalesced
+//              stores: no float atomics).
+//  6. combine: y[t] = bf16(sum of the ybuf rows of token t in selection order,
+//              shared expert last (+ x)): a fixed order, so prefill output does
+//              not depend on scheduling.
 //
 // Warp roles of the GEMM kernel (one CTA per SM, persistent over work items):
 //  warps 0-3   epilogue (TMEM lane quadrant = warp index)
-//  warps 4-11  A producers: each thread dequantises one 32-value group of a row
-//              of both A tiles from the packed codes staged in a small ring
-//  warp 12     TMEM allocation and the single MMA-issuing thread
+//  warps 4-11  A producers in two groups of four warps; group j fills the A
+//              stages of the k-steps g with g % 2 == j, so two k-steps are
+//              dequantised at once.  A thread loads the packed codes of one
+//              32-value group of two rows of both tiles (one group k-step
+//              ahead, into registers) and writes them dequantised, swizzled.
+//  warp 12     TMEM allocation; one elected lane issues the MMAs
 //  warp 13     loads: the B tile of every k-step by TMA (rows of the permuted
-//              token buffer, or of H), and the packed codes by bulk copies
+//              token buffer, or of H) into the k-step ring, and each item's
+//              packed codes into L2 (bulk prefetch) one item ahead
 // Every wait is bounded; a timed-out role records the error and stops waiting.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -48,21 +53,14 @@ cudaError_t launch_prep_tokens(const uint16_t* x, int T, int d, uint32_t flags, 
 
 constexpr int PF_NT = 128;        // token tile = MMA N (max)
 constexpr int PF_BM = 128;        // MMA M
-constexpr int PF_NSA = 3;         // A (dequantised weights) ring stages: produced on chip
-constexpr int PF_NSB = 4;         // B (token rows) ring stages: loaded from memory by TMA
-constexpr int PF_CS = 6;          // packed-code ring stages
+constexpr int PF_NS = 4;          // k-step ring stages: an A tile pair (dequantised on chip)
+                                  // and a B tile (TMA) share one full and one empty barrier
 constexpr int PF_TOKBLK = 256;    // bucketing token block
-// Code stage of one k-step of a tile pair (two groups of 16 packed 16-row
-// tiles), as the 4-D tensor-map boxes land: [tile][group][bytes].
-//  gate/up: Wg lo [8][2][128] @0 | Wu lo @2048 | Wg hi [8][2][64] @4096 | Wu hi @5120
-//           | Wg scales [8][2][32] @6144 | Wu scales @6656
-//  down:    Wd lo [16][2][128] @0 | Wd hi [16][2][64] @4096 | Wd scales [16][2][32] @6144
-constexpr int PF_CODE_STAGE = 7168;
 constexpr int PF_A_TILE = PF_BM * 128;     // one 128 x 64 fp16 tile
 constexpr int PF_A_STAGE = 2 * PF_A_TILE;  // a tile pair
 constexpr int PF_B_STAGE = PF_NT * 128;
 constexpr int PF_THREADS = 14 * 32;
-constexpr int PF_A_THREADS = 256;
+constexpr int PF_A_WARPS = 4;      // warps of one producer group (two groups)
 
 struct PfWs {
   int* counts;      // [E+1]
@@ -74,12 +72,11 @@ struct PfWs {
   int* tokpos;      // [T*(k+1)]
   float* wpos;      // [T*(k+1)]
   __half* H;        // [(T*(k+1) + 128)][Fmax]
-  float* yacc;      // [T][d]
   __half* x16;      // [T][d]
   uint16_t* xn;     // [T][d]
   int* invpos;      // [T*k]: position of entry t*k+j in the buckets (-1: invalid id)
   __half* xperm;    // [T*(k+1)][d]: token rows in bucket order (GEMM1 operand)
-  float* ybuf;      // [T*(k+1)][d]: weighted expert rows (deterministic GEMM2), aliases xperm
+  __half* ybuf;     // [T*(k+1)][d]: weighted expert rows (GEMM2 output), aliases xperm
 };
 
 static size_t pf_max_chunks(const LayerDev& L, int T) {
@@ -99,8 +96,8 @@ size_t prefill_ws_bytes(const LayerDev& L, int T, size_t* parts) {
   parts[6] = pf_max_chunks(L, T) * 16 + 256 + 2 * (R * 4 + 256) + (size_t)T * L.k * 4;
                                                                // chunks, tokpos, wpos, invpos
   parts[7] = (R + PF_NT) * Fmax * 2;                           // H
-  parts[8] = (size_t)T * L.d * 4;                              // yacc
-  parts[9] = R * L.d * 4;                                      // xperm / ybuf
+  parts[8] = 0;                                                // (unused)
+  parts[9] = R * L.d * 2;                                      // xperm / ybuf
   size_t tot = 0;
   for (int i = 0; i < 10; ++i) tot += parts[i];
   return tot;
@@ -125,9 +122,8 @@ static PfWs pf_ws(const LayerDev& L, int T, char* ws, const WsLayout& lay) {
   t += (R * 4 + 255) / 256 * 256;
   p.invpos = reinterpret_cast<int*>(t);
   p.H = reinterpret_cast<__half*>(ws + lay.h);
-  p.yacc = reinterpret_cast<float*>(ws + lay.yacc);
   p.xperm = reinterpret_cast<__half*>(ws + lay.xperm);
-  p.ybuf = reinterpret_cast<float*>(ws + lay.xperm);
+  p.ybuf = reinterpret_cast<__half*>(ws + lay.xperm);
   return p;
 }
 
@@ -274,7 +270,8 @@ __global__ void __launch_bounds__(256) bucket_scatter_kernel(const int32_t* __re
 }
 
 // Token rows in bucket order: xperm[pos] = x16[tokpos[pos]] for the filled
-// positions pos < offsets[E+1] (routed buckets, then the shared bucket).
+// positions pos < offsets[E+1] (routed buckets, then the shared bucket).  One
+// warp per row, 16-byte accesses, four in flight per lane.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __half* __restrict__ x16,
                                                           const int* __restrict__ tokpos,
                                                           const int* __restrict__ offsets, int E,
@@ -282,29 +279,39 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __half* __restri
                                                           int d, Control* ctl) {
   pdl_wait();
   pdl_launch_dependents();
-  const int per = d / 8;
-  const long long n = (long long)offsets[E + 1] * per;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long pos = i / per;
-    const int c = (int)(i - pos * per);
+  const int per = d / 8;   // 16-byte pieces of a row
+  const int lane = threadIdx.x & 31;
+  const int nrows = offsets[E + 1];
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  bool bad = false;
+  for (int pos = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); pos < nrows; pos += nw) {
     int t = tokpos[pos];
     if (t < 0 || t >= T) {
-      record_error(ctl, kErrRange, 0x602);
+      bad = true;
       t = 0;
     }
-    reinterpret_cast<uint4*>(xperm)[i] = reinterpret_cast<const uint4*>(x16 + (size_t)t * d)[c];
+    const uint4* src = reinterpret_cast<const uint4*>(x16 + (size_t)t * d);
+    uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)pos * d);
+    for (int c0 = lane; c0 < per; c0 += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c0 + 32 * u < per) v[u] = src[c0 + 32 * u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c0 + 32 * u < per) dst[c0 + 32 * u] = v[u];
+    }
   }
+  if (bad && lane == 0) record_error(ctl, kErrRange, 0x602);
 }
 
 // ----------------------------------------------------------------- GEMM
 struct PfArgs {
   LayerDev L;
-  int mode;     // 0: gate/up -> H,  1: down -> y_acc (or ybuf)
+  int mode;     // 0: gate/up -> H,  1: down -> ybuf
   int T;
   int Fmax;
   int ppc;      // tile pairs (work items) per chunk
-  int det;      // mode 1: store each position's row to ybuf instead of reducing
   PfWs p;
   Control* ctl;
 };
@@ -384,24 +391,11 @@ struct KSeq {
   }
 };
 
-// Tensor maps: the token (or hidden) rows of the B operand, and the packed
-// codes / scales of the routed experts and of the shared expert viewed as
-// 4-D byte tensors [bytes of a group][group][16-row tile][slot].
+// Tensor map of the B operand: token rows of xperm (mode 0) or hidden rows of
+// H (mode 1).
 struct alignas(64) PfMaps {
   CUtensorMap b;
-  CUtensorMap lo, hi, sc;      // routed experts
-  CUtensorMap slo, shi, ssc;   // shared expert
 };
-
-__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1,
-                                            int c2, int c3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
-      "r"(smem_u32(bar))
-      : "memory");
-}
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
                                             uint64_t* bar) {
@@ -412,32 +406,164 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// One lane: the packed codes and scales of k-step ks of `it` (both tiles of
-// the pair) into a code stage; the layout is given at PF_CODE_STAGE.
+// Read-only global loads that do not allocate in L1 (the packed codes are read
+// once per CTA; reuse across CTAs is served by L2).  Volatile so that they stay
+// ahead of the waits that follow them in program order.
+__device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_nc_u16(const void* p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ void l2_prefetch_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Geometry of the matrices a work item reads: the codes and scales of its
+// expert (slot, or the shared expert), the code bytes of a 16-row tile and the
+// groups along K.
+struct PfGeo {
+  const uint8_t* codes;     // matrix of mode 1 (Wd) / Wg of mode 0
+  const uint16_t* scales;
+  long long up_codes;       // mode 0: Wu codes - Wg codes (bytes)
+  long long up_scales;      // mode 0: Wu scales - Wg scales (elements)
+  int tcb, nG, rows_blk;    // code bytes per 16-row tile, groups along K, 16-row tiles
+};
+
 template <int BITS>
-__device__ __forceinline__ void pf_issue_codes(const PfArgs& a, const PfMaps& mp, const PfItem& it,
-                                               int ks, unsigned char* st, uint64_t* bar) {
-  const CUtensorMap* lo = it.shared ? &mp.slo : &mp.lo;
-  const CUtensorMap* hi = it.shared ? &mp.shi : &mp.hi;
-  const CUtensorMap* sc = it.shared ? &mp.ssc : &mp.sc;
-  const int g0 = 2 * ks;
-  mbar_arrive_expect_tx(bar, 5120 + (BITS == 3 ? 2048 : 0));
+__device__ __forceinline__ PfGeo pf_geo(const PfArgs& a, const PfItem& it) {
+  PfGeo g;
+  constexpr int gb = BITS == 2 ? 8 : 12;
+  const uint8_t* ec = it.shared ? a.L.scodes : a.L.codes + (long long)it.slot * a.L.cbe;
+  const uint16_t* es = it.shared ? a.L.sscales : a.L.scales + (long long)it.slot * a.L.nse;
+  const int nGd = a.L.d / kGroup;
+  const long long tcbd = (long long)nGd * kTileRows * gb;   // Wg / Wu tile bytes
   if (a.mode == 0) {
-    const int tg = 8 * it.pair, tu = it.F / kTileRows + 8 * it.pair;
-    tma_load_4d(st, lo, 0, g0, tg, it.slot, bar);
-    tma_load_4d(st + 2048, lo, 0, g0, tu, it.slot, bar);
-    if (BITS == 3) {
-      tma_load_4d(st + 4096, hi, 0, g0, tg, it.slot, bar);
-      tma_load_4d(st + 5120, hi, 0, g0, tu, it.slot, bar);
-    }
-    tma_load_4d(st + 6144, sc, 0, g0, tg, it.slot, bar);
-    tma_load_4d(st + 6656, sc, 0, g0, tu, it.slot, bar);
+    g.codes = ec;
+    g.scales = es;
+    g.up_codes = (long long)(it.F / kTileRows) * tcbd;
+    g.up_scales = (long long)it.F * nGd;
+    g.tcb = (int)tcbd;
+    g.nG = nGd;
+    g.rows_blk = it.F / kTileRows;
   } else {
-    const int t0 = 16 * it.pair;
-    tma_load_4d(st, lo, 0, g0, t0, it.slot, bar);
-    if (BITS == 3) tma_load_4d(st + 4096, hi, 0, g0, t0, it.slot, bar);
-    tma_load_4d(st + 6144, sc, 0, g0, t0, it.slot, bar);
+    g.codes = ec + 2 * (long long)(it.F / kTileRows) * tcbd;
+    g.scales = es + 2 * (long long)it.F * nGd;
+    g.up_codes = 0;
+    g.up_scales = 0;
+    g.nG = it.F / kGroup;
+    g.tcb = g.nG * kTileRows * gb;
+    g.rows_blk = a.L.d / kTileRows;
   }
+  return g;
+}
+
+// One lane: bring the packed codes and scales an item will read into L2.
+template <int BITS>
+__device__ __forceinline__ void pf_prefetch_item(const PfArgs& a, const PfItem& it) {
+  const PfGeo g = pf_geo<BITS>(a, it);
+  const int per = a.mode == 0 ? 8 : 16;                 // 16-row tiles of a pair, per matrix
+  const int b0 = per * it.pair;
+  const int nb = min(per, g.rows_blk - b0);
+  if (nb <= 0) return;
+  const uint32_t cb = (uint32_t)nb * g.tcb, sb = (uint32_t)nb * g.nG * kTileRows * 2;
+  const uint8_t* c = g.codes + (long long)b0 * g.tcb;
+  const uint16_t* sc = g.scales + (long long)b0 * g.nG * kTileRows;
+  l2_prefetch_bulk(c, cb);
+  l2_prefetch_bulk(sc, sb);
+  if (a.mode == 0) {
+    l2_prefetch_bulk(c + g.up_codes, cb);
+    l2_prefetch_bulk(sc + g.up_scales, sb);
+  }
+}
+
+// The packed codes of one producer thread for one k-step: four units (row rq
+// or rq + 64 of tile 0 or 1, one 32-value group), loaded into registers one
+// group k-step ahead of their use.
+struct PfRaw {
+  uint2 lo[4];
+  uint32_t hi[4];
+  uint32_t sc[4];
+  uint32_t meta;   // bits 0-3: unit u present; bits 4-5: groups in the k-step
+};
+
+// Per-item addresses of a producer thread's four units: the 16-row tile of
+// each unit (codes and scales), computed once per work item.
+struct PfUnits {
+  const uint8_t* tb[4];
+  const uint16_t* sb[4];
+  uint32_t mask;   // units whose rows are inside the matrix
+  int hioff;       // start of the high-bit plane within a tile (bytes)
+  int key;         // the item these addresses belong to (-1: none)
+};
+
+template <int BITS>
+__device__ __forceinline__ void pf_units(const PfArgs& a, const PfItem& it, int rq, PfUnits& U) {
+  const PfGeo g = pf_geo<BITS>(a, it);
+  int blk, dblk, rblk;
+  const uint8_t* mc = g.codes;
+  const uint16_t* ms = g.scales;
+  if (a.mode == 0) {
+    // A-tile rows: four blocks of [16 gate rows, 16 up rows]
+    const int qt = rq >> 5, isu = (rq >> 4) & 1;
+    blk = 8 * it.pair + qt;
+    dblk = 4;
+    rblk = 2;
+    if (isu) {
+      mc += g.up_codes;
+      ms += g.up_scales;
+    }
+  } else {
+    blk = 16 * it.pair + (rq >> 4);
+    dblk = 8;
+    rblk = 4;
+  }
+  uint32_t mask = 0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int b = blk + (u >> 1) * dblk + (u & 1) * rblk;
+    const bool in = b < g.rows_blk && ((u >> 1) == 0 || it.two);
+    U.tb[u] = mc + (long long)(in ? b : 0) * g.tcb;
+    U.sb[u] = ms + (long long)(in ? b : 0) * g.nG * kTileRows;
+    mask |= in ? 1u << u : 0u;
+  }
+  U.mask = mask;
+  U.hioff = g.nG * 128;
+}
+
+template <int BITS>
+__device__ __forceinline__ void pf_load_raw(const PfArgs& a, const KSeq& q, int rq, int gi,
+                                            PfUnits& U, PfRaw& r) {
+  const PfItem& it = q.item_ref();
+  if (U.key != q.s.i) {
+    pf_units<BITS>(a, it, rq, U);
+    U.key = q.s.i;
+  }
+  const int ng = q.ks == it.KS - 1 ? it.ng_last : 2;
+  const int w = (2 * q.ks + gi) * kTileRows + (rq & 15);   // word (group, row) within a tile
+  const uint32_t use = gi < ng ? U.mask : 0u;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    if ((use >> u) & 1u) {
+      r.lo[u] = ldg_nc_v2(U.tb[u] + w * 8);
+      r.hi[u] = BITS == 3 ? ldg_nc_u32(U.tb[u] + U.hioff + w * 4) : 0u;
+      r.sc[u] = ldg_nc_u16(U.sb[u] + w);
+    } else {
+      r.lo[u] = make_uint2(0u, 0u);
+      r.hi[u] = 0u;
+      r.sc[u] = 0u;
+    }
+  }
+  r.meta = ((uint32_t)ng << 4) | use;
 }
 
 // Dequantise chunk m (8 consecutive K values) of one group into fp16.  The
@@ -448,67 +574,44 @@ __device__ __forceinline__ void pf_issue_codes(const PfArgs& a, const PfMaps& mp
 template <int BITS>
 __device__ __forceinline__ uint4 pf_dq_chunk(const uint32_t (&X)[4], const uint32_t (&Y)[4], int m,
                                              __half2 s2) {
+  // fp16 constants as bit patterns (both halves): 4^-m, and the recentring
+  // terms -(1024 + 2) 4^-m (2-bit); for 3 bits the high plane's 2^(2-m) and
+  // -(1024 * 2^(2-m) + 4 + 1024 * 4^-m)
+  constexpr uint32_t kMulR[4] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u};
+  constexpr uint32_t kAddR2[4] = {0xE402E402u, 0xDC08DC08u, 0xD420D420u, 0xCC80CC80u};
+  constexpr uint32_t kMulH[4] = {0x44004400u, 0x40004000u, 0x3C003C00u, 0x38003800u};
+  constexpr uint32_t kAddH[4] = {0xED01ED01u, 0xE882E882u, 0xE444E444u, 0xE028E028u};
   const uint32_t magic = 0x64006400u;
   const uint32_t mask = 0x00030003u << (2 * m);
-  const float mulR = m == 0 ? 1.f : (m == 1 ? 0.25f : (m == 2 ? 0.0625f : 0.015625f));
   uint32_t out[4];
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
     const __half2 R = u32_as_h2(and_or(X[t], mask, magic));
     __half2 v;
     if (BITS == 2) {
-      const float addR = m == 0 ? -1026.f : (m == 1 ? -258.f : (m == 2 ? -66.f : -18.f));
-      v = __hfma2(R, __float2half2_rn(mulR), __float2half2_rn(addR));
+      v = __hfma2(R, u32_as_h2(kMulR[m]), u32_as_h2(kAddR2[m]));
     } else {
-      const float mulH = m == 0 ? 4.f : (m == 1 ? 2.f : (m == 2 ? 1.f : 0.5f));
-      const float addH = m == 0 ? -5124.f : (m == 1 ? -2308.f : (m == 2 ? -1092.f : -532.f));
       const __half2 H = u32_as_h2(and_or(Y[t], 0x00010001u << m, magic));
-      const __half2 tmp = __hfma2(H, __float2half2_rn(mulH), __float2half2_rn(addH));
-      v = __hfma2(R, __float2half2_rn(mulR), tmp);
+      const __half2 tmp = __hfma2(H, u32_as_h2(kMulH[m]), u32_as_h2(kAddH[m]));
+      v = __hfma2(R, u32_as_h2(kMulR[m]), tmp);
     }
     out[t] = h2_as_u32(__hmul2(v, s2));
   }
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
-// One (row, group) unit of an A tile: read its codes and scale from the code
-// stage (zeros when the row or group is outside the matrix).
-template <int BITS>
-__device__ __forceinline__ void pf_read_unit(const unsigned char* cst, bool use, int lo_off,
-                                             int hi_off, int sc_off, uint32_t (&X)[4],
-                                             uint32_t (&Y)[4], __half2& s2) {
-  if (use) {
-    const uint2 lo = *reinterpret_cast<const uint2*>(cst + lo_off);
-    const uint32_t hi = BITS == 3 ? *reinterpret_cast<const uint32_t*>(cst + hi_off) : 0u;
-    s2 = __half2half2(*reinterpret_cast<const __half*>(cst + sc_off));
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      X[t] = __byte_perm(lo.x, lo.y, (uint32_t)t | ((uint32_t)(4 + t) << 8));
-      Y[t] = hi >> (4 * t);
-    }
-  } else {
-    s2 = __float2half2_rn(0.f);
-#pragma unroll
-    for (int t = 0; t < 4; ++t) X[t] = Y[t] = 0u;
-  }
-}
-
 struct PfSmem {
-  size_t a, b, codes, stage_h, bars, holder, total;
+  size_t a, b, bars, holder, total;
 };
 __host__ __device__ inline PfSmem pf_smem() {
   PfSmem m;
   size_t o = 0;
   m.a = o;
-  o += (size_t)PF_NSA * PF_A_STAGE;
+  o += (size_t)PF_NS * PF_A_STAGE;
   m.b = o;
-  o += (size_t)PF_NSB * PF_B_STAGE;
-  m.codes = o;
-  o += (size_t)PF_CS * PF_CODE_STAGE;
-  m.stage_h = o;                       // epilogue staging of H rows: [128 n][64 f] fp16
-  o += (size_t)PF_NT * 64 * 2;
+  o += (size_t)PF_NS * PF_B_STAGE;
   m.bars = o;
-  o += (2 * PF_NSA + 2 * PF_NSB + 2 * PF_CS + 4) * 8;
+  o += (2 * PF_NS + 4) * 8;
   m.holder = o;
   o += 16;
   m.total = o + 1024;   // slack to align the base to 1024
@@ -524,32 +627,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
   const PfSmem m = pf_smem();
   unsigned char* sA = smem + m.a;
   unsigned char* sB = smem + m.b;
-  unsigned char* sC = smem + m.codes;
-  __half* sH = reinterpret_cast<__half*>(smem + m.stage_h);
-  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + m.bars);
-  uint64_t* emptyA = fullA + PF_NSA;
-  uint64_t* fullB = emptyA + PF_NSA;
-  uint64_t* emptyB = fullB + PF_NSB;
-  uint64_t* cfull = emptyB + PF_NSB;
-  uint64_t* cempty = cfull + PF_CS;
-  uint64_t* tfull = cempty + PF_CS;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + m.bars);   // A by 4 warps + B by TMA
+  uint64_t* empty = full + PF_NS;                                  // MMA commit
+  uint64_t* tfull = empty + PF_NS;
   uint64_t* tempty = tfull + 2;
   uint32_t* holder = reinterpret_cast<uint32_t*>(smem + m.holder);
   Control* ctl = a.ctl;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    for (int s = 0; s < PF_NSA; ++s) {
-      mbar_init(&fullA[s], PF_A_THREADS);
-      mbar_init(&emptyA[s], 1);
-    }
-    for (int s = 0; s < PF_NSB; ++s) {
-      mbar_init(&fullB[s], 1);
-      mbar_init(&emptyB[s], 1);
-    }
-    for (int c = 0; c < PF_CS; ++c) {
-      mbar_init(&cfull[c], 1);
-      mbar_init(&cempty[c], PF_A_THREADS);
+    for (int s = 0; s < PF_NS; ++s) {
+      mbar_init(&full[s], PF_A_WARPS + 1);
+      mbar_init(&empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
@@ -561,10 +650,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
     tmem_alloc(holder, 512);
     tmem_relinquish();
   }
-  if (warp == 13 && lane < 7) {   // the seven tensor-map descriptors into the TMA unit's cache
-    const CUtensorMap* maps[7] = {&mp.b, &mp.lo, &mp.hi, &mp.sc, &mp.slo, &mp.shi, &mp.ssc};
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(maps[lane])) : "memory");
-  }
+  if (warp == 13 && lane == 0)   // the B tensor-map descriptor into the TMA unit's cache
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mp.b)) : "memory");
   pdl_wait();
   pdl_launch_dependents();
   tc_fence_before();
@@ -576,133 +663,138 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
 
   if (warp >= 4 && warp < 12) {
     // ------------------------------------------------ A producers (dequant)
-    // Thread = (row r of both tiles, group gi of the k-step).
-    const int ta = tid - 128;
-    const int r = ta >> 1, gi = ta & 1, rr = r & 15;
-    int lo_off, hi_off, sc_off, dlo, dhi, dsc, blk0, dblk;
-    if (a.mode == 0) {
-      // rows of a tile: four blocks of [16 gate rows, 16 up rows]
-      const int qt = r >> 5, isu = (r >> 4) & 1;
-      lo_off = isu * 2048 + qt * 256;
-      hi_off = 4096 + isu * 1024 + qt * 128;
-      sc_off = 6144 + isu * 512 + qt * 64;
-      dlo = 1024, dhi = 512, dsc = 256;
-      blk0 = qt, dblk = 4;   // 16-row feature block within the pair
-    } else {
-      const int q16 = r >> 4;
-      lo_off = q16 * 256;
-      hi_off = 4096 + q16 * 128;
-      sc_off = 6144 + q16 * 64;
-      dlo = 2048, dhi = 1024, dsc = 512;
-      blk0 = q16, dblk = 8;
-    }
-    lo_off += gi * 128 + rr * 8;
-    hi_off += gi * 64 + rr * 4;
-    sc_off += gi * 32 + rr * 2;
-    const int nblk = a.mode == 0 ? 0 : a.L.d / kTileRows;   // mode 0: set per item
-    unsigned char* const adst = sA + r * 128;
-    KSeq cur;
-    cur.init(a, n_items);
-    int cs = 0, sa = 0;
-    uint32_t pc = 0, pa = 0;
-    int g = 0;
-    while (!cur.done) {
-      const PfItem& it = cur.item_ref();
-      const int ng = cur.ks == it.KS - 1 ? it.ng_last : 2;
-      const int rows_blk = a.mode == 0 ? it.F / kTileRows : nblk;
-      const int b0 = (a.mode == 0 ? 8 : 16) * it.pair + blk0;
-      const bool u0 = gi < ng && b0 < rows_blk;
-      const bool u1 = gi < ng && b0 + dblk < rows_blk && it.two;
-      if (ok) ok = mbar_wait(&cfull[cs], pc, ctl, 0x610);
-      uint32_t X0[4], Y0[4], X1[4], Y1[4];
-      __half2 s0, s1;
-      const unsigned char* cst = sC + cs * PF_CODE_STAGE;
-      pf_read_unit<BITS>(cst, u0 && ok, lo_off, hi_off, sc_off, X0, Y0, s0);
-      pf_read_unit<BITS>(cst, u1 && ok, lo_off + dlo, hi_off + dhi, sc_off + dsc, X1, Y1, s1);
-      mbar_arrive(&cempty[cs]);   // code stage read
-      if (++cs == PF_CS) {
-        cs = 0;
-        pc ^= 1u;
-      }
-      uint4 c0[4], c1[4];
+    // Group grp = k-step parity.  Thread = (group gi of the k-step, rows rq and
+    // rq + 64 of both tiles): four 32-value units per k-step, whose packed
+    // codes are loaded one group k-step (two k-steps) ahead.
+    const int grp = (warp - 4) >> 2;
+    const int ta = tid - 128 - 128 * grp;
+    const int rq = ta >> 1, gi = ta & 1;
+    // swizzled 16-byte chunk offsets of this thread's group in a row
+    uint32_t swz[4];
 #pragma unroll
-      for (int mm = 0; mm < 4; ++mm) c0[mm] = pf_dq_chunk<BITS>(X0, Y0, mm, s0);
-#pragma unroll
-      for (int mm = 0; mm < 4; ++mm) c1[mm] = pf_dq_chunk<BITS>(X1, Y1, mm, s1);
-      if (g >= PF_NSA && ok) ok = mbar_wait(&emptyA[sa], pa ^ 1u, ctl, 0x611);
-      if (gi < ng) {
+    for (int mm = 0; mm < 4; ++mm) swz[mm] = (uint32_t)(((4 * gi + mm) ^ (rq & 7)) << 4);
+    unsigned char* const adst = sA + rq * 128;
+    KSeq q;
+    q.init(a, n_items);
+    if (grp == 1 && !q.done) q.advance(a);
+    // Two register buffers alternate: the codes of the group's next k-step
+    // load while the current one is dequantised, and no copy of a buffer
+    // waits on its loads.
+    auto produce = [&](const PfRaw& r, int g) {
+      const int sa = g % PF_NS;
+      if (g >= PF_NS && ok) ok = mbar_wait(&empty[sa], ((g / PF_NS) - 1) & 1, ctl, 0x611);
+      if (gi < (int)(r.meta >> 4)) {
+        // unit u: tile u >> 1 (+16 KB), row rq + 64 (u & 1) (+8 KB); absent
+        // units (rows outside the matrix) are written as zeros
         unsigned char* at = adst + sa * PF_A_STAGE;
 #pragma unroll
-        for (int mm = 0; mm < 4; ++mm) {
-          const int c = 4 * gi + mm;
-          *reinterpret_cast<uint4*>(at + ((c ^ (r & 7)) << 4)) = c0[mm];
-          *reinterpret_cast<uint4*>(at + PF_A_TILE + ((c ^ (r & 7)) << 4)) = c1[mm];
+        for (int u = 0; u < 4; ++u) {
+          uint32_t X[4], Y[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            X[t] = __byte_perm(r.lo[u].x, r.lo[u].y, (uint32_t)t | ((uint32_t)(4 + t) << 8));
+            Y[t] = r.hi[u] >> (4 * t);
+          }
+          const __half2 s2 = __half2half2(__ushort_as_half((unsigned short)r.sc[u]));
+#pragma unroll
+          for (int mm = 0; mm < 4; ++mm)
+            *reinterpret_cast<uint4*>(at + (u >> 1) * PF_A_TILE + (u & 1) * 8192 + swz[mm]) =
+                pf_dq_chunk<BITS>(X, Y, mm, s2);
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(&fullA[sa]);
-      if (++sa == PF_NSA) {
-        sa = 0;
-        pa ^= 1u;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[sa]);
+    };
+    auto skip2 = [&]() {   // this group's next k-step
+      q.advance(a);
+      if (!q.done) q.advance(a);
+    };
+    PfRaw r0, r1;
+    PfUnits U;
+    U.key = -1;
+    bool have0 = !q.done;
+    if (have0) {
+      pf_load_raw<BITS>(a, q, rq, gi, U, r0);
+      skip2();
+    }
+    int g = grp;
+    while (have0) {
+      const bool have1 = !q.done;
+      if (have1) {
+        pf_load_raw<BITS>(a, q, rq, gi, U, r1);
+        skip2();
       }
-      ++g;
-      cur.advance(a);
+      produce(r0, g);
+      g += 2;
+      if (!have1) break;
+      have0 = !q.done;
+      if (have0) {
+        pf_load_raw<BITS>(a, q, rq, gi, U, r0);
+        skip2();
+      }
+      produce(r1, g);
+      g += 2;
     }
   } else if (warp == 13) {
-    // ------------------------------------------------ loads (TMA)
-    if (lane == 0) {
-      KSeq cur, ahead;
-      cur.init(a, n_items);
-      ahead.init(a, n_items);
-      int g = 0, gc = 0, sb = 0, cs = 0;
-      uint32_t pb = 0, pc = 0;
-      while (!cur.done) {
-        // packed codes up to PF_CS k-steps ahead of the B loads
-        while (!ahead.done && gc < g + PF_CS) {
-          if (gc >= PF_CS && ok) ok = mbar_wait(&cempty[cs], pc ^ 1u, ctl, 0x621);
-          pf_issue_codes<BITS>(a, mp, ahead.item_ref(), ahead.ks, sC + cs * PF_CODE_STAGE, &cfull[cs]);
-          if (++cs == PF_CS) {
-            cs = 0;
-            pc ^= 1u;
-          }
-          ahead.advance(a);
-          ++gc;
-        }
-        if (g >= PF_NSB && ok) ok = mbar_wait(&emptyB[sb], pb ^ 1u, ctl, 0x620);
-        mbar_arrive_expect_tx(&fullB[sb], PF_B_STAGE);
-        tma_load_2d(sB + sb * PF_B_STAGE, &mp.b, 64 * cur.ks, cur.item_ref().pos0, &fullB[sb]);
-        if (++sb == PF_NSB) {
-          sb = 0;
-          pb ^= 1u;
-        }
-        cur.advance(a);
-        ++g;
+    // ------------------------------------------------ loads: B by TMA, codes into L2
+    // The whole warp walks the loop; one elected lane issues.
+    const bool leader = elect_one();
+    ItemSeq pfs;
+    pfs.init(a, n_items);
+    PfItem pit;
+    bool have = pfs.get(a, pit);
+    if (have && leader) pf_prefetch_item<BITS>(a, pit);
+    have = have && pfs.get(a, pit);
+    KSeq cur;
+    cur.init(a, n_items);
+    int g = 0, sb = 0;
+    uint32_t pb = 0;
+    while (!cur.done) {
+      if (cur.ks == 0 && g > 0 && have) {   // a new item: codes of the one after it
+        if (leader) pf_prefetch_item<BITS>(a, pit);
+        have = pfs.get(a, pit);
       }
+      if (g >= PF_NS && ok) ok = mbar_wait(&empty[sb], pb ^ 1u, ctl, 0x620);
+      if (leader) {
+        mbar_arrive_expect_tx(&full[sb], PF_B_STAGE);
+        tma_load_2d(sB + sb * PF_B_STAGE, &mp.b, 64 * cur.ks, cur.item_ref().pos0, &full[sb]);
+      }
+      __syncwarp();
+      if (++sb == PF_NS) {
+        sb = 0;
+        pb ^= 1u;
+      }
+      cur.advance(a);
+      ++g;
     }
   } else if (warp == 12) {
-    // ------------------------------------------------ MMA issuer (one thread)
-    if (lane == 0) {
-      const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(sA));
-      const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(sB));
-      ItemSeq seq;
-      seq.init(a, n_items);
-      PfItem it;
-      int sa = 0, sb = 0, la = 0;
-      uint32_t pa = 0, pb = 0;
-      while (seq.get(a, it)) {
-        const int acc = la & 1;
-        if (la >= 2 && ok) ok = mbar_wait(&tempty[acc], ((la >> 1) - 1) & 1, ctl, 0x630);
+    // ------------------------------------------------ MMA issuer
+    // The whole warp walks the loop (its values stay warp-uniform); one
+    // elected lane issues the MMAs and the commits.
+    const bool leader = elect_one();
+    const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(sA));
+    const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(sB));
+    ItemSeq seq;
+    seq.init(a, n_items);
+    PfItem it;
+    int s = 0, la = 0;
+    uint32_t ph = 0;
+    while (seq.get(a, it)) {
+      const int acc = la & 1;
+      if (la >= 2 && ok) ok = mbar_wait(&tempty[acc], ((la >> 1) - 1) & 1, ctl, 0x630);
+      tc_fence_after();
+      const uint32_t idesc = idesc_f16_f32(PF_BM, (it.nv + 15) & ~15);
+      const uint32_t d0 = tmem_base + (uint32_t)(acc * 256), d1 = d0 + 128;
+      const bool two = it.two;
+      for (int ks = 0; ks < it.KS; ++ks) {
+        if (ok) ok = mbar_wait(&full[s], ph, ctl, 0x631);
         tc_fence_after();
-        const uint32_t idesc = idesc_f16_f32(PF_BM, (it.nv + 15) & ~15);
-        const uint32_t d0 = tmem_base + (uint32_t)(acc * 256), d1 = d0 + 128;
-        const bool two = it.two;
-        for (int ks = 0; ks < it.KS; ++ks) {
-          if (ok) ok = mbar_wait(&fullB[sb], pb, ctl, 0x632);
-          if (ok) ok = mbar_wait(&fullA[sa], pa, ctl, 0x631);
-          tc_fence_after();
-          const uint64_t ad = adesc0 + (uint64_t)(sa * (PF_A_STAGE >> 4));
-          const uint64_t bd = bdesc0 + (uint64_t)(sb * (PF_B_STAGE >> 4));
-          const uint32_t first = ks > 0 ? 1u : 0u;
+        const uint64_t ad = adesc0 + (uint64_t)(s * (PF_A_STAGE >> 4));
+        const uint64_t bd = bdesc0 + (uint64_t)(s * (PF_B_STAGE >> 4));
+        const uint32_t first = ks > 0 ? 1u : 0u;
+        const bool full = ks < it.KS - 1 || it.ng_last == 2;
+        if (leader) {
           if (ok) {
             tc_mma_f16(d0, ad, bd, idesc, first);
             tc_mma_f16(d0, ad + 2, bd + 2, idesc, 1u);
@@ -710,7 +802,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
               tc_mma_f16(d1, ad + (PF_A_TILE >> 4), bd, idesc, first);
               tc_mma_f16(d1, ad + (PF_A_TILE >> 4) + 2, bd + 2, idesc, 1u);
             }
-            if (ks < it.KS - 1 || it.ng_last == 2) {
+            if (full) {
               tc_mma_f16(d0, ad + 4, bd + 4, idesc, 1u);
               tc_mma_f16(d0, ad + 6, bd + 6, idesc, 1u);
               if (two) {
@@ -719,20 +811,17 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
               }
             }
           }
-          tc_commit(&emptyA[sa]);
-          tc_commit(&emptyB[sb]);
-          if (++sa == PF_NSA) {
-            sa = 0;
-            pa ^= 1u;
-          }
-          if (++sb == PF_NSB) {
-            sb = 0;
-            pb ^= 1u;
-          }
+          tc_commit(&empty[s]);
         }
-        tc_commit(&tfull[acc]);
-        ++la;
+        __syncwarp();
+        if (++s == PF_NS) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
+      if (leader) tc_commit(&tfull[acc]);
+      __syncwarp();
+      ++la;
     }
   } else {
     // ------------------------------------------------ epilogue (warps 0-3)
@@ -743,24 +832,37 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
     int la = 0;
     while (seq.get(a, it)) {
       const int acc = la & 1;
+      // mode 1: routing weights of this item's columns (lane + 32 c)
+      float wcol[4] = {0.f, 0.f, 0.f, 0.f};
+      if (a.mode == 1) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (lane + 32 * c < it.nv) wcol[c] = a.p.wpos[it.pos0 + lane + 32 * c];
+      }
       if (ok) ok = mbar_wait(&tfull[acc], (la >> 1) & 1, ctl, 0x640);
       tc_fence_after();
       const int n_mma = (it.nv + 15) & ~15;
       const int ntile = it.two ? 2 : 1;
       if (a.mode == 0) {
-        // SwiGLU into the staging tile sH[n][64 f], then coalesced row stores.
-        // TMEM lane 32q + l holds gate row 16q + l (l < 16) or the matching
-        // up row (l >= 16); each step pairs two token columns so that every
-        // lane computes one output.
-        const int fl = 16 * q + (lane & 15);
+        // SwiGLU straight to H.  TMEM lane 32q + l holds gate row 16q + l
+        // (l < 16) or the matching up row (l >= 16); each step pairs two token
+        // columns so that every lane computes one output, and a store
+        // instruction writes two 32-byte row segments of H.
         const int hi = lane >> 4;
         for (int v = 0; v < ntile; ++v) {
           const uint32_t taddr =
               tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * 256 + v * 128);
+          const int fcol = 64 * (2 * it.pair + v) + 16 * q + (lane & 15);
+          const bool fok = ok && fcol < it.F;
+          __half* dst = a.p.H + (size_t)it.pos0 * a.Fmax + fcol;
           for (int c0 = 0; c0 < n_mma; c0 += 32) {
             uint32_t rv[32];
             tmem_ld_32x32b_x32(taddr + c0, rv);
             tmem_ld_wait();
+            if (v == ntile - 1 && c0 + 32 >= n_mma) {
+              tc_fence_before();
+              mbar_arrive(&tempty[acc]);   // TMEM free: the MMA may start item + 2
+            }
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               const float a0 = __uint_as_float(rv[j]), a1 = __uint_as_float(rv[j + 1]);
@@ -768,61 +870,37 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
               const float gv = hi ? got : a0;
               const float up = hi ? a1 : got;
               const float h = __fdividef(gv * up, 1.f + __expf(-gv));
-              sH[(c0 + j + hi) * 64 + fl] = __float2half_rn(h);
+              const int n = c0 + j + hi;
+              if (fok && n < it.nv) dst[(size_t)n * a.Fmax] = __float2half_rn(h);
             }
           }
-          if (v == ntile - 1) {
-            tc_fence_before();
-            mbar_arrive(&tempty[acc]);   // TMEM free: the MMA may start item + 2
-          }
-          named_bar_sync(3, 128);
-          const int fcol = 64 * (2 * it.pair + v) + 2 * lane;
-          if (ok && fcol < it.F) {
-            __half* dst = a.p.H + (size_t)it.pos0 * a.Fmax + fcol;
-            for (int n = q; n < it.nv; n += 4)
-              *reinterpret_cast<uint32_t*>(dst + (size_t)n * a.Fmax) =
-                  *reinterpret_cast<const uint32_t*>(sH + n * 64 + 2 * lane);
-          }
-          named_bar_sync(3, 128);
         }
       } else {
+        // weighted rows of the down projection into ybuf[position][i] (fp16),
+        // one coalesced 64-byte row segment per column and warp
         for (int v = 0; v < ntile; ++v) {
           const uint32_t taddr =
               tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * 256 + v * 128);
           const int i_out = PF_BM * (2 * it.pair + v) + 32 * q + lane;
           const bool wr = i_out < a.L.d && ok;
+          __half* dst = a.p.ybuf + (size_t)it.pos0 * a.L.d + i_out;
           for (int c0 = 0; c0 < n_mma; c0 += 32) {
             uint32_t rv[32];
             tmem_ld_32x32b_x32(taddr + c0, rv);
-            // routing weight and destination of column c0 + lane
-            const int nl = c0 + lane;
-            int tok = 0;
-            float wv = 0.f;
-            if (nl < it.nv) {
-              tok = a.p.tokpos[it.pos0 + nl];
-              wv = a.p.wpos[it.pos0 + nl];
-            }
             tmem_ld_wait();
+            if (v == ntile - 1 && c0 + 32 >= n_mma) {
+              tc_fence_before();
+              mbar_arrive(&tempty[acc]);
+            }
+            const float wl = c0 == 0 ? wcol[0] : (c0 == 32 ? wcol[1] : (c0 == 64 ? wcol[2] : wcol[3]));
             const int jn = min(32, it.nv - c0);
-            if (a.det) {
-              float* dst = a.p.ybuf + (size_t)(it.pos0 + c0) * a.L.d + i_out;
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const float wj = __shfl_sync(0xffffffffu, wv, j);
-                if (j < jn && wr) dst[(size_t)j * a.L.d] = __uint_as_float(rv[j]) * wj;
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const float wj = __shfl_sync(0xffffffffu, wv, j);
-                const int tj = __shfl_sync(0xffffffffu, tok, j);
-                if (j < jn && wr) atomicAdd(a.p.yacc + (size_t)tj * a.L.d + i_out, __uint_as_float(rv[j]) * wj);
-              }
+            for (int j = 0; j < 32; ++j) {
+              const float wj = __shfl_sync(0xffffffffu, wl, j);
+              if (j < jn && wr) dst[(size_t)(c0 + j) * a.L.d] = __float2half_rn(__uint_as_float(rv[j]) * wj);
             }
           }
         }
-        tc_fence_before();
-        mbar_arrive(&tempty[acc]);
       }
       ++la;
     }
@@ -833,76 +911,63 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
   if (warp == 12) tmem_dealloc(tmem_base, 512);
 }
 
-// y = bf16(y_acc (+ x)), four elements per thread.
-__global__ void __launch_bounds__(256) prefill_finalize_kernel(const float* __restrict__ yacc,
-                                                               const uint16_t* __restrict__ x,
-                                                               long long n4, uint32_t flags,
-                                                               uint16_t* __restrict__ y) {
-  pdl_wait();
-  pdl_launch_dependents();
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
-       i += (long long)gridDim.x * blockDim.x) {
-    float4 v = reinterpret_cast<const float4*>(yacc)[i];
-    if (flags & MOE_F_RESIDUAL) {
-      const uint2 xv = reinterpret_cast<const uint2*>(x)[i];
-      v.x += __uint_as_float(xv.x << 16);
-      v.y += __uint_as_float(xv.x & 0xFFFF0000u);
-      v.z += __uint_as_float(xv.y << 16);
-      v.w += __uint_as_float(xv.y & 0xFFFF0000u);
-    }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-    uint2 o;
-    o.x = *reinterpret_cast<uint32_t*>(&lo);
-    o.y = *reinterpret_cast<uint32_t*>(&hi);
-    reinterpret_cast<uint2*>(y)[i] = o;
-  }
-}
-
-// Fixed-order combine (MOE_F_DETERMINISTIC): y[t] = bf16(sum over j = 0..k-1 of
-// ybuf[invpos[t][j]] + ybuf[shared row of t] (+ x[t])), the routed terms in
-// selection order and the shared expert last; every term already carries its
-// routing weight.
-__global__ void __launch_bounds__(256) prefill_finalize_det_kernel(
-    const float* __restrict__ ybuf, const int* __restrict__ invpos, const int* __restrict__ offsets,
+// Combine: y[t] = bf16(sum over j = 0..k-1 of ybuf[invpos[t][j]] + ybuf[shared
+// row of t] (+ x[t])), the routed terms in selection order and the shared
+// expert last, in fp32; every term already carries its routing weight.  The
+// fixed order makes the result independent of scheduling.  One warp per
+// token, 8 elements (16 bytes of fp16) per lane and step.
+__global__ void __launch_bounds__(256) prefill_combine_kernel(
+    const __half* __restrict__ ybuf, const int* __restrict__ invpos, const int* __restrict__ offsets,
     const uint16_t* __restrict__ x, int T, int d, int k, int E, int has_shared, uint32_t flags,
     uint16_t* __restrict__ y) {
   pdl_wait();
   pdl_launch_dependents();
-  const int per = d / 4;
-  const long long n4 = (long long)T * per;
+  const int per = d / 8;
   const int sh0 = offsets[E];
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int t = (int)(i / per), c = (int)(i - (long long)t * per);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const int pos = invpos[(size_t)t * k + j];
-      if (pos < 0) continue;
-      const float4 u = reinterpret_cast<const float4*>(ybuf + (size_t)pos * d)[c];
-      v.x += u.x;
-      v.y += u.y;
-      v.z += u.z;
-      v.w += u.w;
+  const int lane = threadIdx.x & 31;
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nw) {
+    const int mypos = lane < k ? invpos[(size_t)t * k + lane] : -1;
+    for (int c = lane; c < per; c += 32) {
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      for (int j = 0; j <= k; ++j) {
+        int pos;
+        if (j < k) {
+          pos = __shfl_sync(0xffffffffu, mypos, j);
+        } else {
+          if (!has_shared) break;
+          pos = sh0 + t;
+        }
+        if (pos < 0) continue;
+        const uint4 u = reinterpret_cast<const uint4*>(ybuf + (size_t)pos * d)[c];
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(u32_as_h2(w4[e]));
+          v[2 * e] += f.x;
+          v[2 * e + 1] += f.y;
+        }
+      }
+      const size_t i = (size_t)t * per + c;
+      if (flags & MOE_F_RESIDUAL) {
+        const uint4 xv = reinterpret_cast<const uint4*>(x)[i];
+        const uint32_t x4[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[2 * e] += __uint_as_float(x4[e] << 16);
+          v[2 * e + 1] += __uint_as_float(x4[e] & 0xFFFF0000u);
+        }
+      }
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+        o[e] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      reinterpret_cast<uint4*>(y)[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    if (has_shared) {
-      const float4 u = reinterpret_cast<const float4*>(ybuf + (size_t)(sh0 + t) * d)[c];
-      v.x += u.x;
-      v.y += u.y;
-      v.z += u.z;
-      v.w += u.w;
-    }
-    if (flags & MOE_F_RESIDUAL) {
-      const uint2 xv = reinterpret_cast<const uint2*>(x)[i];
-      v.x += __uint_as_float(xv.x << 16);
-      v.y += __uint_as_float(xv.x & 0xFFFF0000u);
-      v.z += __uint_as_float(xv.y << 16);
-      v.w += __uint_as_float(xv.y & 0xFFFF0000u);
-    }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-    uint2 o;
-    o.x = *reinterpret_cast<uint32_t*>(&lo);
-    o.y = *reinterpret_cast<uint32_t*>(&hi);
-    reinterpret_cast<uint2*>(y)[i] = o;
   }
 }
 
@@ -918,9 +983,10 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D fp16 row-major tensor [rows][inner] for tiles of PF_NT rows x 64
-// elements, 128-byte swizzle (the canonical K-major UMMA layout).
-static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+// 2-D 16-bit row-major tensor [rows][inner] (fp16 or bf16: the copy moves
+// bytes) for tiles of 128 rows x 64 elements, 128-byte swizzle (the canonical
+// K-major UMMA layout).
+bool make_map_b16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, rows};
@@ -930,46 +996,6 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 4-D byte tensor [inner bytes][groups][tiles][slots] with the given strides.
-static bool make_map4(CUtensorMap* m, const void* base, uint64_t inner, uint64_t groups,
-                      uint64_t tiles, uint64_t slots, uint64_t s_group, uint64_t s_tile,
-                      uint64_t s_slot, uint32_t box_tiles) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[4] = {inner, groups, tiles, slots};
-  cuuint64_t strides[3] = {s_group, s_tile, s_slot};
-  cuuint32_t box[4] = {(cuuint32_t)inner, 2, box_tiles, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// Maps of one expert set (routed: E slots, or the shared expert: 1 slot).
-// Boxes cover a tile pair: 8 16-row tiles of Wg (and of Wu) in mode 0, 16
-// 16-row tiles of Wd in mode 1.
-static bool make_code_maps(const LayerDev& L, int mode, const uint8_t* codes, const uint16_t* scales,
-                           int F, uint64_t slots, CUtensorMap* lo, CUtensorMap* hi, CUtensorMap* sc) {
-  const int gb = group_bytes(L.bits);
-  const uint64_t cbe = 3ull * F * L.d / kGroup * gb, nse2 = 3ull * F * L.d / kGroup * 2;
-  const uint64_t nG = L.d / kGroup, nGF = F / kGroup;
-  const uint64_t tcb = nG * kTileRows * gb, tcbD = nGF * kTileRows * gb;
-  const uint64_t mcb = (uint64_t)(F / kTileRows) * tcb;
-  const uint64_t sslot = cbe, sslot_s = nse2;   // slot strides (unused when slots == 1)
-  if (mode == 0) {
-    const uint64_t tiles = 2ull * F / kTileRows;
-    return make_map4(lo, codes, 128, nG, tiles, slots, 128, tcb, sslot, 8) &&
-           (L.bits == 2 || make_map4(hi, codes + nG * 128, 64, nG, tiles, slots, 64, tcb, sslot, 8)) &&
-           make_map4(sc, scales, 32, nG, tiles, slots, 32, 32 * nG, sslot_s, 8);
-  }
-  const uint64_t tiles = (uint64_t)L.d / kTileRows;
-  const uint8_t* wd = codes + 2 * mcb;
-  const uint8_t* wds = reinterpret_cast<const uint8_t*>(scales) + 2ull * F * nG * 2;
-  return make_map4(lo, wd, 128, nGF, tiles, slots, 128, tcbD, sslot, 16) &&
-         (L.bits == 2 || make_map4(hi, wd + nGF * 128, 64, nGF, tiles, slots, 64, tcbD, sslot, 16)) &&
-         make_map4(sc, wds, 32, nGF, tiles, slots, 32, 32 * nGF, sslot_s, 16);
 }
 
 template <int BITS>
@@ -988,14 +1014,9 @@ cudaError_t launch_prefill(const LayerDev& L, const uint16_t* x, int T, const in
   PfWs p = pf_ws(L, T, ws, lay);
   const int Fmax = L.F > L.Fs ? L.F : L.Fs;
   const int nblk = (T + PF_TOKBLK - 1) / PF_TOKBLK;
-  const bool det = (flags & MOE_F_DETERMINISTIC) != 0;
   const int has_shared = L.Fs > 0 ? 1 : 0;
   cudaError_t e = launch_prep_tokens(x, T, L.d, flags, p.xn, p.x16, ctl, st);
   if (e != cudaSuccess) return e;
-  if (!det) {
-    e = cudaMemsetAsync(p.yacc, 0, (size_t)T * L.d * sizeof(float), st);
-    if (e != cudaSuccess) return e;
-  }
   e = launch_pdl(bucket_hist_kernel, dim3(nblk), dim3(256), (size_t)L.E * 4, st, ids, T, L.k, L.E,
                  p.blockcnt, ctl);
   if (e != cudaSuccess) return e;
@@ -1013,20 +1034,14 @@ cudaError_t launch_prefill(const LayerDev& L, const uint16_t* x, int T, const in
   PfMaps m0, m1;
   memset(&m0, 0, sizeof m0);
   memset(&m1, 0, sizeof m1);
-  if (!make_map(&m0.b, p.xperm, (uint64_t)L.d, (uint64_t)R) ||
-      !make_map(&m1.b, p.H, (uint64_t)Fmax, (uint64_t)(R + PF_NT)) ||
-      !make_code_maps(L, 0, L.codes, L.scales, L.F, L.E, &m0.lo, &m0.hi, &m0.sc) ||
-      !make_code_maps(L, 1, L.codes, L.scales, L.F, L.E, &m1.lo, &m1.hi, &m1.sc))
-    return cudaErrorInvalidValue;
-  if (L.Fs > 0 && (!make_code_maps(L, 0, L.scodes, L.sscales, L.Fs, 1, &m0.slo, &m0.shi, &m0.ssc) ||
-                   !make_code_maps(L, 1, L.scodes, L.sscales, L.Fs, 1, &m1.slo, &m1.shi, &m1.ssc)))
+  if (!make_map_b16(&m0.b, p.xperm, (uint64_t)L.d, (uint64_t)R) ||
+      !make_map_b16(&m1.b, p.H, (uint64_t)Fmax, (uint64_t)(R + PF_NT)))
     return cudaErrorInvalidValue;
   PfArgs a;
   a.L = L;
   a.T = T;
   a.Fmax = Fmax;
   a.p = p;
-  a.det = det ? 1 : 0;
   a.ctl = ctl;
   a.mode = 0;
   a.ppc = (Fmax + 127) / 128;
@@ -1036,15 +1051,11 @@ cudaError_t launch_prefill(const LayerDev& L, const uint16_t* x, int T, const in
   a.ppc = (L.d + 2 * PF_BM - 1) / (2 * PF_BM);
   e = L.bits == 2 ? launch_gemm<2>(a, m1, st) : launch_gemm<3>(a, m1, st);
   if (e != cudaSuccess) return e;
-  const long long n4 = (long long)T * L.d / 4;
-  int grid = (int)((n4 + 255) / 256);
+  int grid = (T + 7) / 8;
   if (grid > 4 * sm_count()) grid = 4 * sm_count();
-  if (det)
-    return launch_pdl(prefill_finalize_det_kernel, dim3(grid), dim3(256), 0, st,
-                      static_cast<const float*>(p.ybuf), static_cast<const int*>(p.invpos),
-                      static_cast<const int*>(p.offsets), x, T, L.d, L.k, L.E, has_shared, flags, y);
-  return launch_pdl(prefill_finalize_kernel, dim3(grid), dim3(256), 0, st,
-                    static_cast<const float*>(p.yacc), x, n4, flags, y);
+  return launch_pdl(prefill_combine_kernel, dim3(grid), dim3(256), 0, st,
+                    static_cast<const __half*>(p.ybuf), static_cast<const int*>(p.invpos),
+                    static_cast<const int*>(p.offsets), x, T, L.d, L.k, L.E, has_shared, flags, y);
 }
 
 }  // namespace moe

@@ -23,21 +23,23 @@ constexpr float kRmsEps = 1e-6f;
 // ids (largest first) and renormalised weights.  Each lane keeps the best of
 // its own logits (ties: lowest index, as the lane scans upward); a round takes
 // the warp maximum of the keys and the lowest index holding it (two redux
-// instructions), and only the winning lane rescans.
-__device__ void warp_topk(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
-                          float* __restrict__ w, Control* ctl, bool debug) {
+// instructions), and only the winning lane rescans.  NPER >= E / 32 logits per
+// lane.
+template <int NPER>
+__device__ void warp_topk_n(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
+                            float* __restrict__ w, Control* ctl, bool debug) {
   const int lane = threadIdx.x & 31;
   // all loads first (independent, in flight together), checks afterwards
-  float v[32];
+  float v[NPER];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NPER; ++i) {
     const int e = lane + 32 * i;
     v[i] = e < E ? __ldcg(row + e) : 0.f;
   }
-  uint32_t key[32];
+  uint32_t key[NPER];
   bool bad = false;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NPER; ++i) {
     key[i] = order_key(v[i]);
     bad |= (lane + 32 * i < E) && !isfinite(v[i]);
   }
@@ -47,15 +49,15 @@ __device__ void warp_topk(const float* __restrict__ row, int E, int k, int32_t* 
   // wins, equal keys go to the lower index; 0 marks invalid or taken entries
   uint32_t bk = 0u, bi = 0xFFFFFFFFu;
   auto rescan = [&]() {
-    unsigned long long c[32];
+    unsigned long long c[NPER];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < NPER; ++i) {
       const uint32_t e = (uint32_t)(lane + 32 * i);
       const bool ok = ((int)e < E) && !((taken >> i) & 1u);
       c[i] = ok ? ((unsigned long long)key[i] << 32) | (unsigned long long)(~e) : 0ull;
     }
 #pragma unroll
-    for (int half = 16; half >= 1; half >>= 1) {
+    for (int half = NPER / 2; half >= 1; half >>= 1) {
 #pragma unroll
       for (int i = 0; i < half; ++i) c[i] = c[i + half] > c[i] ? c[i + half] : c[i];
     }
@@ -84,6 +86,17 @@ __device__ void warp_topk(const float* __restrict__ row, int E, int k, int32_t* 
   const float ex = lane < k ? expf(my_v - v0) : 0.f;
   const float den = warp_sum(ex);
   if (lane < k) w[lane] = ex / den;
+}
+
+__device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, int k,
+                                          int32_t* __restrict__ ids, float* __restrict__ w,
+                                          Control* ctl, bool debug) {
+  if (E <= 128)
+    warp_topk_n<4>(row, E, k, ids, w, ctl, debug);
+  else if (E <= 512)
+    warp_topk_n<16>(row, E, k, ids, w, ctl, debug);
+  else
+    warp_topk_n<32>(row, E, k, ids, w, ctl, debug);
 }
 
 // --------------------------------------------------------- x (bf16) staging
@@ -258,66 +271,6 @@ __global__ void __launch_bounds__(256) prep_tokens_kernel(const uint16_t* __rest
   }
 }
 
-// fp32 GEMM: logits[T][E] = X[T][d] (bf16) * Wr[E][d]^T + b.
-// 128 x 128 tile, K-step 16, 256 threads, 8 x 8 outputs per thread.
-constexpr int RB_M = 128, RB_N = 128, RB_K = 16;
-__global__ void __launch_bounds__(256) router_gemm_kernel(LayerDev L, const uint16_t* __restrict__ X,
-                                                          int T, float* __restrict__ logits) {
-  __shared__ __align__(16) float As[RB_K][RB_M + 4];
-  __shared__ __align__(16) float Bs[RB_K][RB_N + 4];
-  pdl_wait();
-  pdl_launch_dependents();
-  const int tid = threadIdx.x;
-  const int m0 = blockIdx.y * RB_M, n0 = blockIdx.x * RB_N;
-  const int tx = tid % 16, ty = tid / 16;   // 16 x 16 threads; rows ty+16i, cols tx+16j
-  float acc[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  const int d = L.d;
-  for (int k0 = 0; k0 < d; k0 += RB_K) {
-    // A tile: 128 rows x 16 k (bf16) -> As[k][m]
-    for (int i = tid; i < RB_M * RB_K; i += 256) {
-      int m = i / RB_K, kk = i % RB_K;
-      int gm = m0 + m;
-      float v = 0.f;
-      if (gm < T) v = bf16_bits_to_float(X[(size_t)gm * d + k0 + kk]);
-      As[kk][m] = v;
-    }
-    // B tile: 128 experts x 16 k (fp32) -> Bs[k][n]
-    for (int i = tid; i < RB_N * RB_K; i += 256) {
-      int n = i / RB_K, kk = i % RB_K;
-      int gn = n0 + n;
-      Bs[kk][n] = gn < L.E ? __ldg(L.Wr + (size_t)gn * d + k0 + kk) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < RB_K; ++kk) {
-      float a[8], b[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) a[i] = As[kk][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) b[j] = Bs[kk][tx + 16 * j];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int gm = m0 + ty + 16 * i;
-    if (gm >= T) continue;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      int gn = n0 + tx + 16 * j;
-      if (gn < L.E) logits[(size_t)gm * L.E + gn] = acc[i][j] + (L.bias ? L.bias[gn] : 0.f);
-    }
-  }
-}
-
 __global__ void __launch_bounds__(256) topk_kernel(LayerDev L, const float* __restrict__ logits,
                                                    int T, int32_t* __restrict__ ids,
                                                    float* __restrict__ w, uint32_t flags,
@@ -331,10 +284,9 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerDev L, const float* __re
 }
 
 cudaError_t launch_router_large(const LayerDev& L, const uint16_t* x, int T, uint32_t flags,
-                                float* logits, int32_t* ids, float* w, Control* ctl,
-                                cudaStream_t st) {
-  dim3 grid((L.E + RB_N - 1) / RB_N, (T + RB_M - 1) / RB_M);
-  cudaError_t e = launch_pdl(router_gemm_kernel, grid, dim3(256), 0, st, L, x, T, logits);
+                                float* logits, int32_t* ids, float* w, uint16_t* wsplit,
+                                Control* ctl, cudaStream_t st) {
+  cudaError_t e = launch_router_tc(L, x, T, logits, wsplit, wsplit + (size_t)L.E * L.d, ctl, st);
   if (e != cudaSuccess) return e;
   return launch_pdl(topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, L,
                     static_cast<const float*>(logits), T, ids, w, flags, ctl);

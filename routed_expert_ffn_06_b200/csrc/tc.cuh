@@ -7,6 +7,19 @@
 
 namespace moe {
 
+// One lane of a converged warp (the same lane on every call): the issuer of the
+// warp's tcgen05 / TMA instructions while the whole warp walks the loop, so
+// that the loop's values stay warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ------------------------------------------------------------- TMEM alloc
 // One full warp executes these (.sync.aligned).  The allocated TMEM address
 // (lane 0, first column) is written to *holder in shared memory.

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from routed_expert_ffn_06_b200 import build, moe, synth
-from _util import GpuBlock, assert_close, oracle_check
+from _util import GpuBlock, assert_close, logit_bound, oracle_check
 
 pytestmark = pytest.mark.gpu
 
@@ -41,7 +41,8 @@ def test_tiny_config_prefill(T):
 @pytest.mark.parametrize("bits", [2, 3])
 @pytest.mark.parametrize("shape", [dict(d=128, E=32, F=64, Fs=64, k=4),
                                    dict(d=256, E=64, F=128, Fs=0, k=6),
-                                   dict(d=192, E=40, F=96, Fs=160, k=3)])
+                                   dict(d=192, E=40, F=96, Fs=160, k=3),
+                                   dict(d=160, E=24, F=64, Fs=32, k=2)])
 def test_prefill_small_shapes(bits, shape):
     sh = synth.MoEShape(bits=bits, **shape)
     layer = synth.make_layer(sh, seed=11, device="cuda", bias="normal", bias_std=1.0)
@@ -181,4 +182,26 @@ def test_prefill_full_size_deterministic_matches_sampled_oracle():
     assert torch.equal(y1, y2)
     rows = np.random.default_rng(1).choice(T, 48, replace=False)
     oracle_check(layer, x, logits, ids, w, y1, rows=rows)
+    assert gb.error_word() == (0, 0)
+
+
+@pytest.mark.parametrize("T,d,E", [(9, 64, 16), (300, 96, 40), (1000, 2048, 512)])
+def test_router_large_T_tensor_core(T, d, E):
+    """Routing of a long batch (tensor-core logits, split bf16 router weights):
+    logits within the fp32 bound of the oracle's fp64 logits, selection equal
+    to the oracle's on the device logits, weights summing to one."""
+    sh = synth.MoEShape(d=d, E=E, F=64, Fs=0, k=min(10, E // 2), bits=2)
+    layer = synth.make_layer(sh, seed=T, device="cuda", bias="normal")
+    x = synth.make_tokens(T, d, seed=T + 1, device="cuda")
+    gb = GpuBlock(layer, T)
+    logits, ids, w = gb.route(x)
+    torch.cuda.synchronize()
+    lg = logits.cpu().numpy()
+    OL = oracle.OracleLayer(layer.to("cpu"))
+    xv = x.cpu().double().numpy()
+    ref = OL.router_logits(xv)
+    bound = logit_bound(layer, xv)
+    assert np.all(np.abs(lg - ref) <= bound), float(np.max(np.abs(lg - ref) / bound))
+    assert np.array_equal(oracle.select_topk_f32(lg, sh.k), ids.cpu().numpy())
+    assert np.allclose(w.sum(1).cpu().numpy(), 1.0, atol=1e-5)
     assert gb.error_word() == (0, 0)
