@@ -154,6 +154,27 @@ moe_status moe_expert_ffn_prefill(const moe_layer* layer, const void* x_bf16, in
 moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t T, void* y_bf16,
                              uint32_t flags, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_block_forward for a decode window (0 <= T <= 4) without a caller
+ * workspace: the scratch is a 2 MiB array in the library's device memory, one
+ * per device.  The Strata pages have no counterpart; this is for callers that
+ * cannot allocate or own a workspace (a plain C host without a device
+ * allocator, a step loop that must not call cudaMalloc, which synchronises the
+ * device).
+ *  - Allocates nothing.  The first call on a device (with that device
+ *    current) looks up the array's address with cudaGetSymbolAddress; make
+ *    that first call before any stream capture.
+ *  - The array starts zeroed (module load) and every call leaves its control
+ *    block zeroed again; nothing else has to be initialised.
+ *  - One scratch per device: calls on the same device must be ordered (one
+ *    stream, or events); overlapping calls race on the scratch.
+ *  - Shapes whose workspace (moe_workspace_bytes(layer, T)) exceeds 2 MiB
+ *    return MOE_ERR_WORKSPACE_TOO_SMALL; T > 4 returns
+ *    MOE_ERR_UNSUPPORTED_SHAPE; both before anything is enqueued.
+ *  - Device-side error bits go to the array's control block, which no entry
+ *    point reads back; use moe_block_forward with a workspace to inspect them. */
+moe_status moe_block_forward_noalloc(const moe_layer* layer, const void* x_bf16, int32_t T,
+                                     void* y_bf16, uint32_t flags, void* stream);
+
 const char* moe_status_string(moe_status status);
 
 /* Library build information (a static string). */

@@ -31,7 +31,7 @@ F_DEBUG = 8
 
 EXPORTS = ["moe_workspace_bytes", "moe_workspace_init", "moe_workspace_error", "moe_route_topk",
            "moe_expert_ffn_decode", "moe_expert_ffn_prefill", "moe_block_forward",
-           "moe_status_string", "moe_build_info"]
+           "moe_block_forward_noalloc", "moe_status_string", "moe_build_info"]
 
 
 class MoEError(RuntimeError):
@@ -79,6 +79,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.moe_expert_ffn_prefill.argtypes = [P, vp, i32, vp, vp, vp, vp, vp, u32, vp, sz, vp]
     L.moe_block_forward.restype = st
     L.moe_block_forward.argtypes = [P, vp, i32, vp, u32, vp, sz, vp]
+    L.moe_block_forward_noalloc.restype = st
+    L.moe_block_forward_noalloc.argtypes = [P, vp, i32, vp, u32, vp]
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_status_string.argtypes = [st]
     L.moe_build_info.restype = ctypes.c_char_p
@@ -168,6 +170,13 @@ def moe_block_forward(layer: moe_layer, x, T: int, y, flags: int, ws, stream=Non
     _check(load().moe_block_forward(ctypes.byref(layer), _ptr(x), int(T), _ptr(y), int(flags),
                                     _ptr(ws), ws.numel(), _stream(stream)),
            "moe_block_forward")
+
+
+def moe_block_forward_noalloc(layer: moe_layer, x, T: int, y, flags: int, stream=None):
+    """Decode-window block forward on the library's static device scratch."""
+    _check(load().moe_block_forward_noalloc(ctypes.byref(layer), _ptr(x), int(T), _ptr(y),
+                                            int(flags), _stream(stream)),
+           "moe_block_forward_noalloc")
 
 
 def moe_status_string(status: int) -> str:
