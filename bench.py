@@ -19,6 +19,7 @@ Prints one JSON line (rank 0).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -146,6 +147,33 @@ def measured_peaks():
     except (OSError, KeyError, ValueError):
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                 "src": "fallback"}
+
+
+def sources_sha256() -> str:
+    """Hash of the kernel sources (csrc + the C header)."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "routed_expert_ffn_06_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(f.encode())
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    with open(os.path.join(ROOT, "include", "moe.h"), "rb") as fh:
+        h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(name: str):
+    """DRAM bytes (read + write) per launch of the named kernel group from an
+    ncu capture recorded in profiles/traffic.json; None when the file is missing
+    or the kernel sources changed after the counters were taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            d = json.load(f)[name]
+        if d.get("sources_sha256") != sources_sha256():
+            return None
+        return int(d["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError, TypeError):
+        return None
 
 
 # ------------------------------------------------------------------ decode
@@ -326,7 +354,7 @@ def bench_decode(args, rank, world, local):
                    "weights_gen_s": round(t_gen, 1)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "traffic": None, "peak_src": peaks["src"],
+                     "traffic": measured_traffic("decode_expert_step"), "peak_src": peaks["src"],
                      "kernel": "expert step (decode_gu + decode_dn per moe_expert_ffn_decode call)",
                      "bytes_per_launch": round(exp_bytes / (Gc * nwin)),
                      "us_per_launch_by_T": per_T},
@@ -436,16 +464,18 @@ def bench_prefill(args, rank, world, local):
                    "mma": "tcgen05 kind::f16, fp16 operands (weights dequantised to smem), fp32 TMEM"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                     "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "traffic": measured_traffic("prefill_expert_step"),
                      "peak_src": peaks["src"] + " (bf16 burst; fp16 has the same nominal rate)",
-                     "kernel": "expert step (prep, bucketing, GEMM1, GEMM2, finalize per "
+                     "kernel": "expert step (prep, bucketing, gather, GEMM1, GEMM2, combine per "
                                "moe_expert_ffn_prefill call)",
                      "flops_per_launch": flops, "us_per_launch": round(exp_ms * 1e3, 1)},
         "clocks": clk.summary(),
         "e2e": {"value": round(Ke * T * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * sh.d * 2, "d2h_bytes_per_step": T * sh.d * 2,
                 "steps": Ke, "path": "moe_block_forward via the ctypes binding, pinned host x/y"},
-        "gpu_launches": K * 11,   # router GEMM, top-k, prep, hist, scan, scatter, GEMM1, GEMM2, finalize (+memset)
+        # split router, router GEMM, top-k, prep, hist, scan, scatter, gather, GEMM1, GEMM2, combine
+        "gpu_launches": K * 11,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
