@@ -13,128 +13,9 @@
 // Large T (prefill): a tiled fp32 GEMM writes the logits, then one warp per
 // token selects.
 #include "internal.h"
+#include "select.cuh"
 
 namespace moe {
-
-constexpr float kRmsEps = 1e-6f;
-
-// ---------------------------------------------------------------- selection
-// One warp selects top_k of E (E <= 1024) logits of one token and writes the
-// ids (largest first) and renormalised weights.  Each lane keeps the best of
-// its own logits (ties: lowest index, as the lane scans upward); a round takes
-// the warp maximum of the keys and the lowest index holding it (two redux
-// instructions), and only the winning lane rescans.  NPER >= E / 32 logits per
-// lane.
-template <int NPER>
-__device__ void warp_topk_n(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
-                            float* __restrict__ w, Control* ctl, bool debug) {
-  const int lane = threadIdx.x & 31;
-  // all loads first (independent, in flight together), checks afterwards
-  float v[NPER];
-#pragma unroll
-  for (int i = 0; i < NPER; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = e < E ? __ldcg(row + e) : 0.f;
-  }
-  uint32_t key[NPER];
-  bool bad = false;
-#pragma unroll
-  for (int i = 0; i < NPER; ++i) {
-    key[i] = order_key(v[i]);
-    bad |= (lane + 32 * i < E) && !isfinite(v[i]);
-  }
-  if (debug && bad) record_error(ctl, kErrNonFinite, 0x100);
-  uint32_t taken = 0;
-  // lane-local best by a depth-5 tree over (key << 32 | ~index): larger key
-  // wins, equal keys go to the lower index; 0 marks invalid or taken entries
-  uint32_t bk = 0u, bi = 0xFFFFFFFFu;
-  auto rescan = [&]() {
-    unsigned long long c[NPER];
-#pragma unroll
-    for (int i = 0; i < NPER; ++i) {
-      const uint32_t e = (uint32_t)(lane + 32 * i);
-      const bool ok = ((int)e < E) && !((taken >> i) & 1u);
-      c[i] = ok ? ((unsigned long long)key[i] << 32) | (unsigned long long)(~e) : 0ull;
-    }
-#pragma unroll
-    for (int half = NPER / 2; half >= 1; half >>= 1) {
-#pragma unroll
-      for (int i = 0; i < half; ++i) c[i] = c[i + half] > c[i] ? c[i + half] : c[i];
-    }
-    if (c[0] == 0ull) {
-      bk = 0u;
-      bi = 0xFFFFFFFFu;
-    } else {
-      bk = (uint32_t)(c[0] >> 32);
-      bi = ~(uint32_t)(c[0] & 0xFFFFFFFFull);
-    }
-  };
-  rescan();
-  float my_v = 0.f;
-  for (int j = 0; j < k; ++j) {
-    const uint32_t mk = __reduce_max_sync(0xffffffffu, bi == 0xFFFFFFFFu ? 0u : bk);
-    const uint32_t win = __reduce_min_sync(0xffffffffu, (bi != 0xFFFFFFFFu && bk == mk) ? bi : 0xFFFFFFFFu);
-    const uint32_t u = (mk & 0x80000000u) ? (mk & 0x7FFFFFFFu) : ~mk;
-    if (lane == j) my_v = __uint_as_float(u);
-    if (lane == 0) ids[j] = static_cast<int32_t>(win);
-    if ((win & 31u) == (uint32_t)lane) {
-      taken |= 1u << (win >> 5);
-      rescan();
-    }
-  }
-  const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
-  const float ex = lane < k ? expf(my_v - v0) : 0.f;
-  const float den = warp_sum(ex);
-  if (lane < k) w[lane] = ex / den;
-}
-
-__device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, int k,
-                                          int32_t* __restrict__ ids, float* __restrict__ w,
-                                          Control* ctl, bool debug) {
-  if (E <= 128)
-    warp_topk_n<4>(row, E, k, ids, w, ctl, debug);
-  else if (E <= 512)
-    warp_topk_n<16>(row, E, k, ids, w, ctl, debug);
-  else
-    warp_topk_n<32>(row, E, k, ids, w, ctl, debug);
-}
-
-// --------------------------------------------------------- x (bf16) staging
-// Loads T token rows into shared memory as bf16 bits (16-byte loads, all
-// tokens in one pass); with PRENORM replaces them by
-// bf16(x / sqrt(mean(x^2) + eps)), computed in fp32.  red: >= T floats.
-__device__ void stage_tokens(const uint16_t* __restrict__ x, int T, int d, bool prenorm,
-                             uint16_t* xs, float* red) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  if (prenorm) {
-    for (int t = tid; t < T; t += nt) red[t] = 0.f;
-    __syncthreads();
-  }
-  const int per = d / 8;
-  for (int i = tid; i < T * per; i += nt) {
-    const uint4 v = reinterpret_cast<const uint4*>(x)[i];
-    reinterpret_cast<uint4*>(xs)[i] = v;
-    if (prenorm) {
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-      float ss = 0.f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float a = __uint_as_float(w4[j] << 16), b = __uint_as_float(w4[j] & 0xFFFF0000u);
-        ss += a * a + b * b;
-      }
-      atomicAdd(&red[i / per], ss);
-    }
-  }
-  __syncthreads();
-  if (prenorm) {
-    for (int i = tid; i < T * d; i += nt) {
-      const float inv = rsqrtf(red[i / d] / (float)d + kRmsEps);
-      __nv_bfloat16 bv = __float2bfloat16_rn(bf16_bits_to_float(xs[i]) * inv);
-      xs[i] = *reinterpret_cast<uint16_t*>(&bv);
-    }
-    __syncthreads();
-  }
-}
 
 // ------------------------------------------------------------- small T router
 // grid: ceil(E/4) CTAs of 16 warps; four warps per expert row, each a quarter

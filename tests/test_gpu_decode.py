@@ -150,3 +150,17 @@ def test_decode_3bit_stack_layer_prenorm_residual():
     logits, ids, w = gb.route(x, flags)
     y = gb.decode(x, ids, w, flags)
     oracle_check(layer, x, logits, ids, w, y, flags=flags)
+
+
+@pytest.mark.parametrize("T", [4, 8])
+def test_decode_wide_model(T):
+    """d = 4096 (the largest supported model width), 4- and 8-token windows,
+    3-bit: routing and outputs match the oracle."""
+    sh = synth.MoEShape(d=4096, E=32, F=64, Fs=64, k=4, bits=3)
+    layer = synth.make_layer(sh, seed=12, device="cuda", bias="normal")
+    x = synth.make_tokens(T, sh.d, seed=T, device="cuda")
+    gb = GpuBlock(layer, T)
+    logits, ids, w = gb.route(x)
+    y = gb.decode(x, ids, w)
+    oracle_check(layer, x, logits, ids, w, y)
+    assert gb.error_word() == (0, 0)
