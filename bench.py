@@ -39,7 +39,7 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=None)
     p.add_argument("--warmup", type=int, default=None)
-    p.add_argument("--workload", default="decode", choices=["decode", "prefill", "stack"])
+    p.add_argument("--workload", default="decode", choices=["decode", "prefill", "stack", "mix"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--layers", type=int, default=32, help="independent layer copies rotated")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -493,6 +493,43 @@ def bench_prefill(args, rank, world, local):
 
 
 # ------------------------------------------------------------------- stack
+def _stack_layers(wl, rank, dev):
+    from routed_expert_ffn_06_b200 import synth
+    return [synth.make_layer(wl["shape"], seed=rank * 1000, layer=l, device=dev, bias=wl["bias"],
+                             slot=wl["slot"]) for l in range(wl["layers"])]
+
+
+def _stack_bytes_per_step(structs, x, T, ws, stream):
+    """Algorithmic HBM bytes of one decode step through the stack: every
+    layer's router (E x d fp32), its unique selected experts and the shared
+    expert, and the window in and out; the routing is taken from an eager pass
+    over the same input."""
+    import torch
+
+    from routed_expert_ffn_06_b200 import moe
+    L0 = structs[0]
+    eb = _expert_bytes_struct(L0)
+    ids = torch.empty(T, L0.top_k, dtype=torch.int32, device=x.device)
+    wts = torch.empty(T, L0.top_k, dtype=torch.float32, device=x.device)
+    y = [torch.empty_like(x), torch.empty_like(x)]
+    tot, src = 0, x
+    flags = moe.F_PRENORM | moe.F_RESIDUAL
+    for l, L in enumerate(structs):
+        moe.moe_route_topk(L, src, T, flags, None, ids, wts, ws, stream)
+        stream.synchronize()
+        U = int(torch.unique(ids).numel())
+        tot += L.n_experts * L.d_model * 4 + (U + 1) * eb + 2 * T * L.d_model * 2
+        moe.moe_block_forward(L, src, T, y[l % 2], flags, ws, stream)
+        src = y[l % 2]
+    stream.synchronize()
+    return tot
+
+
+def _expert_bytes_struct(L) -> int:
+    gb = 8 if L.bits == 2 else 12
+    return 3 * L.ffn * L.d_model // 32 * (gb + 2)
+
+
 def bench_stack(args, rank, world, local):
     """48 routed-MoE layers, 3-bit (~34 GB), Zipf profile, frequency-ordered
     slots, 4 tokens per step, x <- x + MoE(RMSNorm(x)); a step is one pass of
@@ -508,8 +545,7 @@ def bench_stack(args, rank, world, local):
     K = args.steps if args.steps is not None else wl["steps"]
     W = args.warmup if args.warmup is not None else 5
     t_gen = time.time()
-    layers = [synth.make_layer(sh, seed=rank * 1000, layer=l, device=dev, bias=wl["bias"],
-                               slot=wl["slot"]) for l in range(NLy)]
+    layers = _stack_layers(wl, rank, dev)
     t_gen = time.time() - t_gen
     structs = [moe.make_layer_struct(l) for l in layers]
     ws = moe.alloc_workspace(structs[0], T)
@@ -519,8 +555,8 @@ def bench_stack(args, rank, world, local):
     flags = moe.F_PRENORM | moe.F_RESIDUAL
     stream = torch.cuda.Stream(device=dev)
 
-    def enqueue(s):
-        src = x0[s % G]
+    def enqueue(s, src=None):
+        src = x0[s % G] if src is None else src
         for l in range(NLy):
             dst = bufs[l % 2]
             moe.moe_block_forward(structs[l], src, T, dst, flags, ws, stream)
@@ -530,6 +566,7 @@ def bench_stack(args, rank, world, local):
         for s in range(2):
             enqueue(s)
     stream.synchronize()
+    step_bytes = _stack_bytes_per_step(structs, x0[0], T, ws, stream)
     graphs = []
     for s in range(G):
         g = torch.cuda.CUDAGraph()
@@ -556,9 +593,28 @@ def bench_stack(args, rank, world, local):
     st, code = moe.moe_workspace_error(ws, stream)
     if st != 0:
         raise RuntimeError(f"device error word {code:#x}")
-    eb = sh.codes_bytes + sh.n_scales * 2
-    # unique experts per layer are data dependent: estimate bytes from one step's routing
-    return {
+    # end to end: the window from pinned host memory, 48 layers, back to the host
+    xh = x0[0].cpu().pin_memory()
+    yh = torch.empty(T, sh.d, dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(x0[0])
+    Ke = min(K, 64)
+    barrier(world)
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for s in range(Ke):
+            xd.copy_(xh, non_blocking=True)
+            enqueue(s, xd)
+            yh.copy_(bufs[(NLy - 1) % 2], non_blocking=True)
+        f1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
+    peaks = measured_peaks()
+    achieved = step_bytes / (ms / K / 1e3) / 1e9
+    eb = _expert_bytes_struct(structs[0])
+    res = {
         "metric": METRIC, "value": round(K * T * world / (ms / 1e3), 1), "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms / K, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
@@ -566,11 +622,122 @@ def bench_stack(args, rank, world, local):
         "config": {"workload": "decode 48-layer stack of routed-MoE blocks: d=2048, 512 experts "
                                "ffn=512 + shared, top-10, 3-bit g32, Zipf profile, "
                                "frequency-ordered slots, 4 tokens/step, pre-norm + residual",
+                   "tokens_per_step": T,
                    "weights_gb": round(NLy * (sh.E * eb + eb + sh.E * sh.d * 4) / 1e9, 2),
-                   "l2": "inputs larger than L2", "weights_gen_s": round(t_gen, 1),
-                   "parallelism": f"replicas x{world}"},
+                   "l2": "inputs larger than L2 (34 GB of weights per step)",
+                   "weights_gen_s": round(t_gen, 1), "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": None, "peak_src": peaks["src"],
+                     "kernel": "one step: 48 x (router, gate/up, down)",
+                     "bytes_per_launch": step_bytes},
         "clocks": clk.summary(),
+        "e2e": {"value": round(Ke * T * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * sh.d * 2, "d2h_bytes_per_step": T * sh.d * 2,
+                "steps": Ke, "path": "48 x moe_block_forward via the ctypes binding, pinned host x/y"},
         "gpu_launches": K * NLy * 3,
+    }
+    return res
+
+
+def bench_mix(args, rank, world, local):
+    """48 routed-MoE layers, 3-bit: a 32,768-token prompt read as 4 chunks of
+    8192 tokens (each chunk through all 48 layers), then 512 decode steps of 4
+    tokens; every 64 decode steps each layer's expert ranking is re-drawn (the
+    router bias permuted), the packed slot layout staying as it was."""
+    import torch
+
+    from routed_expert_ffn_06_b200 import moe, synth
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    moe.load()
+    wl = synth.WORKLOADS["mix"]
+    sh, T, NLy = wl["shape"], wl["T"], wl["layers"]
+    C, NC = wl["chunk"], wl["chunks"]
+    DS = args.steps if args.steps is not None else wl["decode_steps"]
+    drift = wl["drift_every"]
+    W = args.warmup if args.warmup is not None else 3
+    t_gen = time.time()
+    layers = _stack_layers(wl, rank, dev)
+    t_gen = time.time() - t_gen
+    structs = [moe.make_layer_struct(l) for l in layers]
+    ws = moe.alloc_workspace(structs[0], C)
+    flags = moe.F_PRENORM | moe.F_RESIDUAL
+    stream = torch.cuda.Stream(device=dev)
+    biases = [[l.router_bias.clone()] + [synth.permute_profile(l, seed=rank * 1000, epoch=e + 1)
+                                          for e in range(DS // drift + 1)] for l in layers]
+    chunks = [synth.make_tokens(C, sh.d, seed=rank * 1000 + 21, step=c, device=dev) for c in range(NC)]
+    cb = [torch.empty(C, sh.d, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    G = 16
+    wins = [synth.make_tokens(T, sh.d, seed=rank * 1000 + 22, step=s, device=dev) for s in range(G)]
+    wb = [torch.empty(T, sh.d, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+
+    def run_stack(src, bufs, n):
+        for l in range(NLy):
+            moe.moe_block_forward(structs[l], src, n, bufs[l % 2], flags, ws, stream)
+            src = bufs[l % 2]
+
+    def set_epoch(e):
+        for l in range(NLy):
+            layers[l].router_bias.copy_(biases[l][e], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(W):
+            run_stack(chunks[0], cb, C)
+            run_stack(wins[0], wb, T)
+    stream.synchronize()
+    graphs = []
+    for s in range(G):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run_stack(wins[s], wb, T)
+        graphs.append(g)
+    barrier(world)
+    torch.cuda.synchronize()
+    p0, p1, d1 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            set_epoch(0)
+            p0.record(stream)
+            for c in range(NC):
+                run_stack(chunks[c], cb, C)
+            p1.record(stream)
+            for s in range(DS):
+                if s % drift == 0:
+                    set_epoch(s // drift)
+                graphs[s % G].replay()
+            d1.record(stream)
+        stream.synchronize()
+    barrier(world)
+    ms_pf = max_over_ranks(p0.elapsed_time(p1), world)
+    ms_dec = max_over_ranks(p1.elapsed_time(d1), world)
+    st, code = moe.moe_workspace_error(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device error word {code:#x}")
+    ntok = NC * C + DS * T
+    ms = ms_pf + ms_dec
+    peaks = measured_peaks()
+    flops = 2.0 * NC * C * (sh.k + 1) * 3 * sh.F * sh.d * NLy
+    eb = _expert_bytes_struct(structs[0])
+    return {
+        "metric": METRIC, "value": round(ntok * world / (ms / 1e3), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": DS, "warmup": W, "ms_per_step": round(ms_dec / DS, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic (seeded; random-init weights of the stated architecture)",
+        "config": {"workload": "48-layer 3-bit stack: 32,768-token prompt as 4 x 8192 chunks, then "
+                               "512 decode steps of 4 tokens, expert ranking re-drawn every 64 steps",
+                   "tokens": ntok, "weights_gb": round(NLy * (sh.E * eb + eb + sh.E * sh.d * 4) / 1e9, 2),
+                   "l2": "inputs larger than L2 (34 GB of weights)",
+                   "weights_gen_s": round(t_gen, 1), "parallelism": f"replicas x{world}"},
+        "prefill_tokens_per_s": round(NC * C * world / (ms_pf / 1e3), 1),
+        "decode_tokens_per_s": round(DS * T * world / (ms_dec / 1e3), 1),
+        "roofline": {"bound": "tensor", "achieved": round(flops / (ms_pf / 1e3) / 1e12, 1),
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": round(flops / (ms_pf / 1e3) / 1e12 / peaks["bf16_tflops_sustained"], 4),
+                     "traffic": None, "peak_src": peaks["src"] + " (bf16 sustained)",
+                     "kernel": "prefill phase: 4 chunks x 48 layers (expert GEMM FLOPs)"},
+        "clocks": clk.summary(),
+        "gpu_launches": NC * NLy * 11 + DS * NLy * 3,
     }
 
 
@@ -621,6 +788,8 @@ def main():
             res = bench_decode(args, rank, world, local)
         elif args.workload == "prefill":
             res = bench_prefill(args, rank, world, local)
+        elif args.workload == "mix":
+            res = bench_mix(args, rank, world, local)
         else:
             res = bench_stack(args, rank, world, local)
         if rank == 0 and res is not None:
