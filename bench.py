@@ -57,10 +57,18 @@ def dist_init():
 
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:   # host-only ranks (the oracle arm, tests)
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     return rank, world, local
+
+
+def _reduce_device():
+    import torch.distributed as dist
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
 
 
 def barrier(world):
@@ -74,7 +82,7 @@ def max_over_ranks(v: float, world: int) -> float:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_reduce_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -84,7 +92,7 @@ def sum_over_ranks(v: float, world: int) -> float:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_reduce_device())
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
 
@@ -743,37 +751,71 @@ def bench_mix(args, rank, world, local):
 
 # --------------------------------------------------------------- reference
 def run_reference(args, rank, world):
-    """The fp64 oracle on the host cores, same workload and metric."""
+    """The fp64 oracle on the host cores, on the same workload, metric and unit
+    as our arm (a bounded sample of it per step)."""
     if rank != 0:
         return None
     import oracle
     from routed_expert_ffn_06_b200 import synth
-    wl = synth.WORKLOADS["decode"]
-    layer = synth.make_layer(wl["shape"], seed=0, device="cpu", bias=wl["bias"], slot=wl["slot"])
-    OL = oracle.OracleLayer(layer)
-    K = args.steps if args.steps is not None else 5
-    W = args.warmup if args.warmup is not None else 1
-    W = min(W, 3)
-    K = min(K, 20)
+    K = min(args.steps if args.steps is not None else 5, 20)
+    W = min(args.warmup if args.warmup is not None else 1, 3)
+    if args.workload == "prefill":
+        wl = synth.WORKLOADS["prefill"]
+        layer = synth.make_layer(wl["shape"], seed=0, device="cpu", bias=wl["bias"],
+                                 bias_std=wl["bias_std"], slot=wl["slot"])
+        OL = oracle.OracleLayer(layer)
+        x = synth.make_tokens(wl["T"], wl["shape"].d, seed=3, step=0)
+        per = 16   # tokens of the 8192 chunk per step
 
-    def step(s):
-        for i, T in enumerate(DECODE_WINDOWS):
-            OL.block_forward(synth.make_tokens(T, wl["shape"].d, seed=7, step=s * 4 + i))
+        def step(s):
+            OL.block_forward(x, rows=list(range((s * per) % wl["T"], (s * per) % wl["T"] + per)))
+        workload = ("prefill chunk single layer: 8192 tokens, d=2048, 512 experts ffn=512 + "
+                    "shared ffn=512, top-10, 2-bit g32, router bias N(0,0.5)")
+        sample = f"{per} of the chunk's tokens per step"
+        tok = per
+    elif args.workload in ("stack", "mix"):
+        wl = synth.WORKLOADS["decode_stack"]
+        nl = 2   # layers of the stack per step (the oracle is far too slow for 48)
+        layers = [oracle.OracleLayer(synth.make_layer(wl["shape"], seed=0, layer=l, device="cpu",
+                                                      bias=wl["bias"], slot=wl["slot"]))
+                  for l in range(nl)]
+
+        import torch
+
+        def step(s):
+            x = synth.make_tokens(wl["T"], wl["shape"].d, seed=9, step=s)
+            for OL in layers:
+                r = OL.block_forward(x, flags=oracle.PRENORM | oracle.RESIDUAL)
+                x = torch.from_numpy(r["y"]).to(torch.bfloat16)
+        workload = ("decode 48-layer stack of routed-MoE blocks, 3-bit, 4 tokens/step, pre-norm + "
+                    "residual")
+        sample = f"{nl} of the 48 layers per step, scaled to 48"
+        tok = wl["T"] * nl / 48.0
+    else:
+        wl = synth.WORKLOADS["decode"]
+        layer = synth.make_layer(wl["shape"], seed=0, device="cpu", bias=wl["bias"], slot=wl["slot"])
+        OL = oracle.OracleLayer(layer)
+
+        def step(s):
+            for i, T in enumerate(DECODE_WINDOWS):
+                OL.block_forward(synth.make_tokens(T, wl["shape"].d, seed=7, step=s * 4 + i))
+        workload = ("decode single layer: d=2048, 512 experts ffn=512 + shared ffn=512, top-10, "
+                    "2-bit g32, Zipf(1.1); windows T=1,2,3,4 per step")
+        sample = f"{K} steps of 4 windows (10 tokens)"
+        tok = sum(DECODE_WINDOWS)
     for s in range(W):
         step(s)
     t0 = time.perf_counter()
     for s in range(K):
         step(W + s)
     dt = time.perf_counter() - t0
-    v = K * sum(DECODE_WINDOWS) / dt
+    v = K * tok / dt
     return {"metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": round(1e3 * dt / K, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "impl": "reference",
-            "config": {"workload": "decode single layer: d=2048, 512 experts ffn=512 + shared, "
-                                   "top-10, 2-bit g32, Zipf(1.1); windows T=1,2,3,4 per step"},
+            "data": "synthetic", "impl": "reference", "config": {"workload": workload},
             "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": oracle.num_threads(),
-                             "kind": "oracle", "sample": f"{K} steps of 4 windows (10 tokens)"},
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
