@@ -334,6 +334,52 @@ __device__ __forceinline__ void gu_issue(const LayerDev& L, const ExpList* list,
   }
 }
 
+// Warp-wide copy of `bytes` (a multiple of 16, both ends 16-byte aligned) from
+// global to shared memory, 16 bytes per lane and instruction (cp.async: many
+// small pieces in flight without going through the bulk-copy unit).
+__device__ __forceinline__ void warp_cp_async(void* dst, const void* src, uint32_t bytes) {
+  const int lane = threadIdx.x & 31;
+  for (uint32_t o = (uint32_t)lane * 16; o < bytes; o += 512)
+    cp_async16(static_cast<unsigned char*>(dst) + o, static_cast<const unsigned char*>(src) + o, 16);
+}
+// Wait until at most n of this thread's cp.async groups are pending (n <= 3).
+__device__ __forceinline__ void cp_async_wait_upto(int n) {
+  if (n <= 0)
+    cp_async_wait<0>();
+  else if (n == 1)
+    cp_async_wait<1>();
+  else if (n == 2)
+    cp_async_wait<2>();
+  else
+    cp_async_wait<3>();
+}
+
+// Piece p (groups 8p .. 8p+np-1) of gate/up item (u, tile) into a stage, by
+// the whole warp: one cp.async group.
+template <int BITS>
+__device__ __forceinline__ void gu_copy(const LayerDev& L, const ExpList* list, int u, int tile,
+                                        int p, unsigned char* st, Control* ctl) {
+  const int d = L.d, nG = d / kGroup;
+  const int g0 = kGuPiece * p, np = min(kGuPiece, nG - g0);
+  const ExpSrc src = expert_src(L, list, u, ctl);
+  const long long tcb = (long long)nG * kTileRows * group_bytes(BITS);
+  const long long mcb = mat_codes_bytes(src.F, d, BITS);
+  const long long msc = (long long)src.F * nG;
+  const uint32_t blo = np * kTileRows * 8, bhi = BITS == 3 ? np * kTileRows * 4 : 0;
+  const uint32_t bsc = np * kTileRows * 2;
+  const size_t LO = kGuPiece * kTileRows * 8, HI = BITS == 3 ? kGuPiece * kTileRows * 4 : 0;
+#pragma unroll
+  for (int mat = 0; mat < 2; ++mat) {
+    const uint8_t* tb = src.codes + (mat ? mcb : 0) + tile * tcb;
+    unsigned char* so = st + mat * (LO + HI);
+    warp_cp_async(so, tb + g0 * kTileRows * 8, blo);
+    if (BITS == 3) warp_cp_async(so + LO, tb + (long long)nG * kTileRows * 8 + g0 * kTileRows * 4, bhi);
+    const uint16_t* sb = src.scales + (mat ? msc : 0) + (long long)tile * kTileRows * nG;
+    warp_cp_async(st + 2 * (LO + HI) + mat * kGuPiece * kTileRows * 2, sb + g0 * kTileRows, bsc);
+  }
+  cp_async_commit();
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(kGuWarps * 32, 1)
     decode_gu_kernel(LayerDev L, const uint16_t* __restrict__ x, int T,
@@ -437,32 +483,27 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1)
   const int q_items = my_items > quad ? (my_items - 1 - quad) / nquads + 1 : 0;
   const int total = q_items * ppw;           // this warp's (item, piece) sequence
   unsigned char* wst = smem + m.stages + (size_t)warp * spw * m.stage_bytes;
-  uint64_t* wbar = bars + warp * spw;
   const size_t LO = kGuPiece * kTileRows * 8, HI = BITS == 3 ? kGuPiece * kTileRows * 4 : 0;
   const size_t hwst = hw_expert_halves(Fmax, T);
 
-  auto issue = [&](int q) {   // sequence index q -> (item li, piece wq + 4*j)
+  auto issue = [&](int q) {   // sequence index q -> (item li, piece wq + 4*j); whole warp
     const int li = q / ppw, p = wq + 4 * (q % ppw);
     const int it = quad + li * nquads;
     int u, tile;
     gu_item(L, blockIdx.x + it * gridDim.x, Fs16, F16, &u, &tile);
-    const int s = q % spw;
-    gu_issue<BITS>(L, list, u, tile, p, wst + (size_t)s * m.stage_bytes, &wbar[s], ctl);
+    gu_copy<BITS>(L, list, u, tile, p, wst + (size_t)(q % spw) * m.stage_bytes, ctl);
   };
-  if (lane == 0)
-    for (int q = 0; q < spw && q < total; ++q) issue(q);
+  for (int q = 0; q < spw && q < total; ++q) issue(q);
   int issued = spw < total ? spw : total;
 
-  // A wait that runs out marks the warp failed: it stops reading stages but
-  // still takes every quad barrier, so no warp is left waiting.
-  bool ok = true;
   int seq = 0;
   for (int li = 0; li < q_items; ++li) {
     float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j < ppw; ++j, ++seq) {
       const int s = seq % spw, p = wq + 4 * j;
-      if (ok) ok = mbar_wait(&wbar[s], (seq / spw) & 1, ctl, 0x401);
-      if (ok) {
+      cp_async_wait_upto(issued - 1 - seq);   // this piece's group has landed
+      __syncwarp();
+      {
         const unsigned char* st = wst + (size_t)s * m.stage_bytes;
         const __half* scg = reinterpret_cast<const __half*>(st + 2 * (LO + HI));
         const __half* scu = scg + kGuPiece * kTileRows;
@@ -484,10 +525,7 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1)
       __syncwarp();
       // the stage is free again: refill it with the piece spw steps ahead
       if (issued < total) {
-        if (lane == 0 && ok) {
-          fence_proxy_async_smem();
-          issue(issued);
-        }
+        issue(issued);
         ++issued;
       }
     }
@@ -518,10 +556,7 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1)
       }
     }
   }
-  // no copy may still be landing in this warp's stages when the CTA exits
-  if (lane == 0)
-    for (int q = issued > spw ? issued - spw : 0; q < issued; ++q)
-      mbar_wait(&wbar[q % spw], (q / spw) & 1, ctl, 0x403);
+  cp_async_wait<0>();   // no copy may still be landing in this warp's stages
 }
 
 // ------------------------------------------------------------------- down
