@@ -65,7 +65,8 @@ constexpr int PF_A_WARPS = 4;      // warps of one producer group (two groups)
 struct PfWs {
   int* counts;      // [E+1]
   int* misc;        // [16]: misc[0] = number of chunks
-  int* offsets;     // [E+2]
+  int* offsets;     // [E+2]: padded bucket offsets (internal positions)
+  int* uoffsets;    // [E+2]: bucket offsets without padding (user-visible)
   int* entries;     // [T*k]
   int* blockcnt;    // [nblk][E]
   int4* chunks;     // [maxC]
@@ -79,6 +80,14 @@ struct PfWs {
   __half* ybuf;     // [T*(k+1)][d]: weighted expert rows (GEMM2 output), aliases xperm
 };
 
+// Internal positions: every bucket starts at a multiple of PF_PAD rows (so that
+// whole 32-row blocks of a chunk stay inside its bucket); the padding rows
+// carry token -1.
+constexpr int PF_PAD = 32;
+static size_t pf_rows(const LayerDev& L, int T) {
+  return (size_t)T * (L.k + 1) + (size_t)PF_PAD * (L.E + 1);
+}
+
 static size_t pf_max_chunks(const LayerDev& L, int T) {
   return (size_t)T * L.k / PF_NT + L.E + (T + PF_NT - 1) / PF_NT + 2;
 }
@@ -86,11 +95,11 @@ static size_t pf_max_chunks(const LayerDev& L, int T) {
 size_t prefill_ws_bytes(const LayerDev& L, int T, size_t* parts) {
   const int Fmax = L.F > L.Fs ? L.F : L.Fs;
   const size_t nblk = ((size_t)T + PF_TOKBLK - 1) / PF_TOKBLK;
-  const size_t R = (size_t)T * (L.k + 1);
+  const size_t R = pf_rows(L, T);
   parts[0] = (size_t)T * L.d * 2;                              // xn
   parts[1] = (size_t)T * L.d * 2;                              // x16
   parts[2] = (size_t)(L.E + 1 + 16) * 4;                       // counts + misc
-  parts[3] = (size_t)(L.E + 2) * 4;                            // offsets
+  parts[3] = 2 * (size_t)(L.E + 2) * 4;                        // offsets, uoffsets
   parts[4] = (size_t)T * L.k * 4;                              // entries
   parts[5] = nblk * L.E * 4;                                   // blockcnt
   parts[6] = pf_max_chunks(L, T) * 16 + 256 + 2 * (R * 4 + 256) + (size_t)T * L.k * 4;
@@ -110,13 +119,14 @@ static PfWs pf_ws(const LayerDev& L, int T, char* ws, const WsLayout& lay) {
   p.counts = reinterpret_cast<int*>(ws + lay.counts);
   p.misc = p.counts + L.E + 1;
   p.offsets = reinterpret_cast<int*>(ws + lay.offsets);
+  p.uoffsets = p.offsets + (L.E + 2);
   p.entries = reinterpret_cast<int*>(ws + lay.entries);
   p.blockcnt = reinterpret_cast<int*>(ws + lay.blockcnt);
   char* t = ws + lay.tiles;
   p.chunks = reinterpret_cast<int4*>(t);
   t += (pf_max_chunks(L, T) * 16 + 255) / 256 * 256;
   p.tokpos = reinterpret_cast<int*>(t);
-  const size_t R = (size_t)T * (L.k + 1);
+  const size_t R = pf_rows(L, T);
   t += (R * 4 + 255) / 256 * 256;
   p.wpos = reinterpret_cast<float*>(t);
   t += (R * 4 + 255) / 256 * 256;
@@ -186,7 +196,7 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(int* __restrict__ blo
                                                            const int32_t* __restrict__ slot, PfWs p,
                                                            int* __restrict__ user_offsets,
                                                            Control* ctl) {
-  __shared__ int cnt[2048], off[2048], nch[2048], wt[33];
+  __shared__ int cnt[2048], off[2048], poff[2048], nch[2048], wt[33];
   pdl_wait();
   pdl_launch_dependents();
   const int tid = threadIdx.x;
@@ -203,15 +213,19 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(int* __restrict__ blo
   __syncthreads();
   for (int e = tid; e <= E; e += blockDim.x) {
     off[e] = cnt[e];
+    poff[e] = (cnt[e] + PF_PAD - 1) / PF_PAD * PF_PAD;
     nch[e] = (cnt[e] + PF_NT - 1) / PF_NT;
   }
   __syncthreads();
   block_excl_scan(off, E + 1, wt);
+  block_excl_scan(poff, E + 1, wt);
   const int nchunks = block_excl_scan(nch, E + 1, wt);
   for (int e = tid; e <= E; e += blockDim.x) {
     p.counts[e] = cnt[e];
-    p.offsets[e] = off[e];
+    p.offsets[e] = poff[e];
+    p.uoffsets[e] = off[e];
     if (user_offsets) user_offsets[e] = off[e];
+    for (int r = cnt[e]; r % PF_PAD; ++r) p.tokpos[poff[e] + r] = -1;   // padding rows
     // chunk record: (bucket, first position, rows, weight slot of the bucket)
     int s = 0;
     if (e < E && cnt[e] > 0) {
@@ -222,10 +236,11 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(int* __restrict__ blo
       }
     }
     for (int c = 0; c * PF_NT < cnt[e]; ++c)
-      p.chunks[nch[e] + c] = make_int4(e, off[e] + c * PF_NT, min(PF_NT, cnt[e] - c * PF_NT), s);
+      p.chunks[nch[e] + c] = make_int4(e, poff[e] + c * PF_NT, min(PF_NT, cnt[e] - c * PF_NT), s);
   }
   if (tid == 0) {
-    p.offsets[E + 1] = off[E] + cnt[E];
+    p.offsets[E + 1] = poff[E] + (cnt[E] + PF_PAD - 1) / PF_PAD * PF_PAD;
+    p.uoffsets[E + 1] = off[E] + cnt[E];
     p.misc[0] = nchunks;
   }
 }
@@ -253,10 +268,11 @@ __global__ void __launch_bounds__(256) bucket_scatter_kernel(const int32_t* __re
     }
     int rank = __popc(bits[e * 8 + (lt >> 5)] & ((1u << (lt & 31)) - 1u));
     for (int wd = 0; wd < (lt >> 5); ++wd) rank += __popc(bits[e * 8 + wd]);
-    const int pos = p.offsets[e] + p.blockcnt[(size_t)blockIdx.x * E + e] + rank;
-    p.entries[pos] = i;
+    const int before = p.blockcnt[(size_t)blockIdx.x * E + e] + rank;
+    const int pos = p.offsets[e] + before, upos = p.uoffsets[e] + before;
+    p.entries[upos] = i;
     p.invpos[i] = pos;
-    if (user_entries) user_entries[pos] = i;
+    if (user_entries) user_entries[upos] = i;
     p.tokpos[pos] = t;
     p.wpos[pos] = w[i];
   }
@@ -270,8 +286,9 @@ __global__ void __launch_bounds__(256) bucket_scatter_kernel(const int32_t* __re
 }
 
 // Token rows in bucket order: xperm[pos] = x16[tokpos[pos]] for the filled
-// positions pos < offsets[E+1] (routed buckets, then the shared bucket).  One
-// warp per row, 16-byte accesses, four in flight per lane.
+// positions pos < offsets[E+1] (routed buckets, then the shared bucket; the
+// padding rows are skipped).  One warp per row, 16-byte accesses, four in
+// flight per lane.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __half* __restrict__ x16,
                                                           const int* __restrict__ tokpos,
                                                           const int* __restrict__ offsets, int E,
@@ -286,7 +303,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __half* __restri
   bool bad = false;
   for (int pos = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); pos < nrows; pos += nw) {
     int t = tokpos[pos];
-    if (t < 0 || t >= T) {
+    if (t < 0) continue;   // padding row
+    if (t >= T) {
       bad = true;
       t = 0;
     }
@@ -395,7 +413,25 @@ struct KSeq {
 // H (mode 1).
 struct alignas(64) PfMaps {
   CUtensorMap b;
+  CUtensorMap st;   // epilogue output: H (mode 0, box 64 x 32) or ybuf (mode 1, box 128 x 32)
 };
+
+// 32 output rows of one tile (staged in shared memory) to global memory by TMA.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
                                             uint64_t* bar) {
@@ -600,8 +636,9 @@ __device__ __forceinline__ uint4 pf_dq_chunk(const uint32_t (&X)[4], const uint3
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
+constexpr int PF_OUT_STAGE = 32 * 128 * 2;   // 32 rows x 128 fp16 (mode 1); mode 0 uses 32 x 64
 struct PfSmem {
-  size_t a, b, bars, holder, total;
+  size_t a, b, out, bars, holder, total;
 };
 __host__ __device__ inline PfSmem pf_smem() {
   PfSmem m;
@@ -610,6 +647,8 @@ __host__ __device__ inline PfSmem pf_smem() {
   o += (size_t)PF_NS * PF_A_STAGE;
   m.b = o;
   o += (size_t)PF_NS * PF_B_STAGE;
+  m.out = o;                       // epilogue staging: two 32-row blocks
+  o += 2 * (size_t)PF_OUT_STAGE;
   m.bars = o;
   o += (2 * PF_NS + 4) * 8;
   m.holder = o;
@@ -627,6 +666,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
   const PfSmem m = pf_smem();
   unsigned char* sA = smem + m.a;
   unsigned char* sB = smem + m.b;
+  unsigned char* sOut = smem + m.out;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + m.bars);   // A by 4 warps + B by TMA
   uint64_t* empty = full + PF_NS;                                  // MMA commit
   uint64_t* tfull = empty + PF_NS;
@@ -650,8 +690,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
     tmem_alloc(holder, 512);
     tmem_relinquish();
   }
-  if (warp == 13 && lane == 0)   // the B tensor-map descriptor into the TMA unit's cache
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mp.b)) : "memory");
+  if (warp == 13 && lane < 2)   // the tensor-map descriptors into the TMA unit's cache
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(lane ? &mp.st : &mp.b))
+                 : "memory");
   pdl_wait();
   pdl_launch_dependents();
   tc_fence_before();
@@ -825,11 +866,28 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
     }
   } else {
     // ------------------------------------------------ epilogue (warps 0-3)
+    // Each 32-column block of an accumulator tile becomes 32 output rows,
+    // staged in shared memory (two buffers) and written by one TMA store; the
+    // rows past the chunk's tokens are padding rows of the same bucket.
     const int q = warp;
     ItemSeq seq;
     seq.init(a, n_items);
     PfItem it;
-    int la = 0;
+    int la = 0, cc = 0;
+    // free a staging buffer (the store issued from it two blocks ago has read it)
+    auto claim = [&]() {
+      if (tid == 0 && cc >= 2) bulk_wait_read<1>();
+      named_bar_sync(3, 128);
+    };
+    auto release = [&](int x0, int row0) {
+      fence_proxy_async_smem();
+      named_bar_sync(3, 128);
+      if (tid == 0) {
+        tma_store_2d(&mp.st, sOut + (cc & 1) * PF_OUT_STAGE, x0, row0);
+        bulk_commit();
+      }
+      ++cc;
+    };
     while (seq.get(a, it)) {
       const int acc = la & 1;
       // mode 1: routing weights of this item's columns (lane + 32 c)
@@ -843,67 +901,48 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
       tc_fence_after();
       const int n_mma = (it.nv + 15) & ~15;
       const int ntile = it.two ? 2 : 1;
-      if (a.mode == 0) {
-        // SwiGLU straight to H.  TMEM lane 32q + l holds gate row 16q + l
-        // (l < 16) or the matching up row (l >= 16); each step pairs two token
-        // columns so that every lane computes one output, and a store
-        // instruction writes two 32-byte row segments of H.
-        const int hi = lane >> 4;
-        for (int v = 0; v < ntile; ++v) {
-          const uint32_t taddr =
-              tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * 256 + v * 128);
-          const int fcol = 64 * (2 * it.pair + v) + 16 * q + (lane & 15);
-          const bool fok = ok && fcol < it.F;
-          __half* dst = a.p.H + (size_t)it.pos0 * a.Fmax + fcol;
-          for (int c0 = 0; c0 < n_mma; c0 += 32) {
-            uint32_t rv[32];
-            tmem_ld_32x32b_x32(taddr + c0, rv);
-            tmem_ld_wait();
-            if (v == ntile - 1 && c0 + 32 >= n_mma) {
-              tc_fence_before();
-              mbar_arrive(&tempty[acc]);   // TMEM free: the MMA may start item + 2
-            }
+      for (int v = 0; v < ntile; ++v) {
+        const uint32_t taddr =
+            tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * 256 + v * 128);
+        for (int c0 = 0; c0 < n_mma; c0 += 32) {
+          uint32_t rv[32];
+          tmem_ld_32x32b_x32(taddr + c0, rv);
+          tmem_ld_wait();
+          if (v == ntile - 1 && c0 + 32 >= n_mma) {
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);   // TMEM free: the MMA may start item + 2
+          }
+          claim();
+          __half* so = reinterpret_cast<__half*>(sOut + (cc & 1) * PF_OUT_STAGE);
+          if (a.mode == 0) {
+            // SwiGLU: TMEM lane 32q + l holds gate row 16q + l (l < 16) or the
+            // matching up row (l >= 16); a step pairs two token columns so that
+            // every lane computes one output.  Stage [32 rows][64 f].
+            const int hi = lane >> 4, fl = 16 * q + (lane & 15);
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               const float a0 = __uint_as_float(rv[j]), a1 = __uint_as_float(rv[j + 1]);
               const float got = __shfl_xor_sync(0xffffffffu, hi ? a0 : a1, 16);
               const float gv = hi ? got : a0;
               const float up = hi ? a1 : got;
-              const float h = __fdividef(gv * up, 1.f + __expf(-gv));
-              const int n = c0 + j + hi;
-              if (fok && n < it.nv) dst[(size_t)n * a.Fmax] = __float2half_rn(h);
+              so[(j + hi) * 64 + fl] = __float2half_rn(__fdividef(gv * up, 1.f + __expf(-gv)));
             }
-          }
-        }
-      } else {
-        // weighted rows of the down projection into ybuf[position][i] (fp16),
-        // one coalesced 64-byte row segment per column and warp
-        for (int v = 0; v < ntile; ++v) {
-          const uint32_t taddr =
-              tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * 256 + v * 128);
-          const int i_out = PF_BM * (2 * it.pair + v) + 32 * q + lane;
-          const bool wr = i_out < a.L.d && ok;
-          __half* dst = a.p.ybuf + (size_t)it.pos0 * a.L.d + i_out;
-          for (int c0 = 0; c0 < n_mma; c0 += 32) {
-            uint32_t rv[32];
-            tmem_ld_32x32b_x32(taddr + c0, rv);
-            tmem_ld_wait();
-            if (v == ntile - 1 && c0 + 32 >= n_mma) {
-              tc_fence_before();
-              mbar_arrive(&tempty[acc]);
-            }
+            release(64 * (2 * it.pair + v), it.pos0 + c0);
+          } else {
+            // weighted rows of the down projection: stage [32 rows][128 d]
             const float wl = c0 == 0 ? wcol[0] : (c0 == 32 ? wcol[1] : (c0 == 64 ? wcol[2] : wcol[3]));
-            const int jn = min(32, it.nv - c0);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float wj = __shfl_sync(0xffffffffu, wl, j);
-              if (j < jn && wr) dst[(size_t)(c0 + j) * a.L.d] = __float2half_rn(__uint_as_float(rv[j]) * wj);
+              so[j * 128 + 32 * q + lane] = __float2half_rn(__uint_as_float(rv[j]) * wj);
             }
+            release(PF_BM * (2 * it.pair + v), it.pos0 + c0);
           }
         }
       }
       ++la;
     }
+    if (tid == 0) bulk_wait<0>();   // every output row written before the CTA leaves
   }
   tc_fence_before();
   __syncthreads();
@@ -986,6 +1025,21 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2-D 16-bit row-major tensor [rows][inner] (fp16 or bf16: the copy moves
 // bytes) for tiles of 128 rows x 64 elements, 128-byte swizzle (the canonical
 // K-major UMMA layout).
+// 2-D 16-bit row-major tensor [rows][inner], box [box_rows][box_inner], no
+// swizzle (the epilogue's output stores).
+static bool make_map_b16_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                               uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map_b16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
   auto fn = encode_fn();
   if (!fn) return false;
@@ -1026,7 +1080,7 @@ cudaError_t launch_prefill(const LayerDev& L, const uint16_t* x, int T, const in
   e = launch_pdl(bucket_scatter_kernel, dim3(nblk), dim3(256), (size_t)L.E * 32, st, ids, w, T, L.k,
                  L.E, has_shared, p, entries_out);
   if (e != cudaSuccess) return e;
-  const size_t R = (size_t)T * (L.k + 1);
+  const size_t R = pf_rows(L, T);
   e = launch_pdl(gather_rows_kernel, dim3(4 * sm_count()), dim3(256), 0, st,
                  static_cast<const __half*>(p.x16), static_cast<const int*>(p.tokpos),
                  static_cast<const int*>(p.offsets), L.E, T, p.xperm, L.d, ctl);
@@ -1035,7 +1089,9 @@ cudaError_t launch_prefill(const LayerDev& L, const uint16_t* x, int T, const in
   memset(&m0, 0, sizeof m0);
   memset(&m1, 0, sizeof m1);
   if (!make_map_b16(&m0.b, p.xperm, (uint64_t)L.d, (uint64_t)R) ||
-      !make_map_b16(&m1.b, p.H, (uint64_t)Fmax, (uint64_t)(R + PF_NT)))
+      !make_map_b16(&m1.b, p.H, (uint64_t)Fmax, (uint64_t)(R + PF_NT)) ||
+      !make_map_b16_plain(&m0.st, p.H, (uint64_t)Fmax, (uint64_t)(R + PF_NT), 64, 32) ||
+      !make_map_b16_plain(&m1.st, p.ybuf, (uint64_t)L.d, (uint64_t)R, 128, 32))
     return cudaErrorInvalidValue;
   PfArgs a;
   a.L = L;
