@@ -107,7 +107,10 @@ typedef struct {
 } moe_layer;
 
 /* Bytes of workspace the calls below need for up to max_tokens tokens
- * (0 on invalid arguments). */
+ * (0 on invalid arguments).  The decode path (moe_route_topk with T <= 8,
+ * moe_expert_ffn_decode, moe_block_forward with T <= 4) uses only a leading
+ * part of the layout and accepts any workspace at least that large; the
+ * prefill path needs the full size. */
 size_t moe_workspace_bytes(const moe_layer* layer, int32_t max_tokens);
 
 /* Zero a workspace (enqueued on stream).  Needed once after allocation. */

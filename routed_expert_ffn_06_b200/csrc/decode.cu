@@ -10,7 +10,7 @@
 //  * decode_gu: work item = (expert u, 16-row tile of Wg and Wu).  A quad of
 //    four warps shares an item: each warp takes pieces of 16 quantisation
 //    groups of the K = d contraction, streams them into its own shared-memory
-//    stages with bulk async copies, dequantises the 2/3-bit codes straight into
+//    stages with warp-wide cp.async, dequantises the 2/3-bit codes straight into
 //    mma.sync A fragments (LOP3 + HFMA2: no shared-memory round trip for the
 //    fp16 weights) and multiplies them with the window's tokens (B fragments;
 //    n = 8 covers T <= 8).  The quad adds its partial sums through shared
@@ -22,8 +22,8 @@
 //    experts, then the CTA adds the warps in a fixed order (deterministic, no
 //    atomics) and writes y (bf16, optional residual).
 // The shared expert is expert u = 0 with weight 1 for every token.
-// Each warp owns its stages and fills them itself, so every mbarrier wait
-// targets the stage's current phase.
+// Each warp owns its stages and fills them itself (gate/up: cp.async groups;
+// down: bulk copies on per-stage mbarriers, every wait on the current phase).
 #include "internal.h"
 #include "tc.cuh"
 
@@ -31,7 +31,7 @@ namespace moe {
 
 constexpr int kMaxExp = kMaxDecodeT * 16 + 1;   // window entries + shared
 constexpr int kGuWarps = 16;                 // four quads
-constexpr int kDnWarps = 8;
+constexpr int kDnWarps = 16;
 
 struct ExpList {
   int n;                       // experts in the list (shared first when present)
@@ -260,7 +260,7 @@ __device__ __forceinline__ ExpSrc expert_src(const LayerDev& L, const ExpList* s
 // expert's hidden vector (2*F*T bytes) in one piece.
 __host__ __device__ inline size_t hw_expert_halves(int Fmax, int T) { return (size_t)Fmax * T; }
 
-constexpr int kGuPiece = 8;                  // groups per piece of a gate/up item
+constexpr int kGuPiece = 16;                 // groups per piece of a gate/up item
 struct GuSmem {
   size_t bars, list, first, xs, corr, part, stages, total, stage_bytes;
   int spw;                                   // stages per warp
@@ -309,31 +309,6 @@ __device__ __forceinline__ void gu_item(const LayerDev& L, int i, int Fs16, int 
   }
 }
 
-// Bulk-copy piece p (groups 16p .. 16p+np-1) of gate/up item (u, tile) into a
-// stage (one lane).
-template <int BITS>
-__device__ __forceinline__ void gu_issue(const LayerDev& L, const ExpList* list, int u, int tile,
-                                         int p, unsigned char* st, uint64_t* bar, Control* ctl) {
-  const int d = L.d, nG = d / kGroup;
-  const int g0 = kGuPiece * p, np = min(kGuPiece, nG - g0);
-  const ExpSrc src = expert_src(L, list, u, ctl);
-  const long long tcb = (long long)nG * kTileRows * group_bytes(BITS);
-  const long long mcb = mat_codes_bytes(src.F, d, BITS);
-  const long long msc = (long long)src.F * nG;
-  const uint32_t blo = np * kTileRows * 8, bhi = BITS == 3 ? np * kTileRows * 4 : 0;
-  const uint32_t bsc = np * kTileRows * 2;
-  const size_t LO = kGuPiece * kTileRows * 8, HI = BITS == 3 ? kGuPiece * kTileRows * 4 : 0;
-  mbar_arrive_expect_tx(bar, 2 * (blo + bhi + bsc));
-  for (int mat = 0; mat < 2; ++mat) {
-    const uint8_t* tb = src.codes + (mat ? mcb : 0) + tile * tcb;
-    unsigned char* so = st + mat * (LO + HI);
-    bulk_g2s(so, tb + g0 * kTileRows * 8, blo, bar);
-    if (BITS == 3) bulk_g2s(so + LO, tb + (long long)nG * kTileRows * 8 + g0 * kTileRows * 4, bhi, bar);
-    const uint16_t* sb = src.scales + (mat ? msc : 0) + (long long)tile * kTileRows * nG;
-    bulk_g2s(st + 2 * (LO + HI) + mat * kGuPiece * kTileRows * 2, sb + g0 * kTileRows, bsc, bar);
-  }
-}
-
 // Warp-wide copy of `bytes` (a multiple of 16, both ends 16-byte aligned) from
 // global to shared memory, 16 bytes per lane and instruction (cp.async: many
 // small pieces in flight without going through the bulk-copy unit).
@@ -354,7 +329,7 @@ __device__ __forceinline__ void cp_async_wait_upto(int n) {
     cp_async_wait<3>();
 }
 
-// Piece p (groups 8p .. 8p+np-1) of gate/up item (u, tile) into a stage, by
+// Piece p (groups kGuPiece*p onwards) of gate/up item (u, tile) into a stage, by
 // the whole warp: one cp.async group.
 template <int BITS>
 __device__ __forceinline__ void gu_copy(const LayerDev& L, const ExpList* list, int u, int tile,

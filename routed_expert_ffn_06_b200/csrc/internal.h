@@ -47,6 +47,7 @@ struct WsLayout {
   size_t yacc;       // (unused, zero bytes)
   size_t xperm;      // prefill: fp16 [T*(k+1)][d]: xperm (GEMM1 operand), then ybuf (GEMM2 output)
   size_t wsplit;     // T > decode window: router weights as bf16 hi and lo [2][E][d]
+  size_t decode_total;   // bytes the decode path needs (a prefix of the layout)
   size_t total;
 };
 WsLayout ws_layout(const LayerDev& L, int T);

@@ -90,6 +90,7 @@ moe_status from_cuda(cudaError_t e) {
 
 // Common preamble of every compute entry point.
 moe_status preamble(const moe_layer* layer, int32_t T, const void* x, void* ws, size_t ws_bytes,
+                    bool decode_path,
                     LayerDev* L, WsLayout* lay) {
   moe_status s = validate_layer(layer);
   if (s != MOE_OK) return s;
@@ -97,7 +98,7 @@ moe_status preamble(const moe_layer* layer, int32_t T, const void* x, void* ws, 
   if (!aligned16(x) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_MISALIGNED;
   *L = to_dev(layer);
   *lay = ws_layout(*L, T);
-  if (ws_bytes < lay->total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < (decode_path ? lay->decode_total : lay->total)) return MOE_ERR_WORKSPACE_TOO_SMALL;
   return MOE_OK;
 }
 }  // namespace
@@ -122,6 +123,7 @@ WsLayout ws_layout(const LayerDev& L, int T) {
   o += align256(Tn * L.k * sizeof(float));
   w.hw = o;
   o += align256(decode_hw_bytes(L, T < kMaxDecodeT ? (int)Tn : kMaxDecodeT));
+  w.decode_total = o;   // the decode path (router for T <= 8, decode step) uses no more
   if (T > 0) {
     size_t parts[16];
     prefill_ws_bytes(L, T, parts);
@@ -195,7 +197,7 @@ moe_status moe_route_topk(const moe_layer* layer, const void* x_bf16, int32_t T,
   if (!topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
   if (flags & ~(MOE_F_PRENORM | MOE_F_RESIDUAL | MOE_F_DETERMINISTIC | MOE_F_DEBUG))
     return MOE_ERR_INVALID_ARG;
-  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, &L, &lay);
+  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, T <= kMaxDecodeT, &L, &lay);
   if (s != MOE_OK) return s;
   if ((s = check_device()) != MOE_OK) return s;
   if (T == 0) return MOE_OK;
@@ -227,7 +229,7 @@ moe_status moe_expert_ffn_decode(const moe_layer* layer, const void* x_bf16, int
   if (flags & ~(MOE_F_PRENORM | MOE_F_RESIDUAL | MOE_F_DETERMINISTIC | MOE_F_DEBUG))
     return MOE_ERR_INVALID_ARG;
   if (T > kMaxDecodeT) return MOE_ERR_UNSUPPORTED_SHAPE;
-  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, &L, &lay);
+  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, true, &L, &lay);
   if (s != MOE_OK) return s;
   if (!aligned16(y_bf16)) return MOE_ERR_MISALIGNED;
   if (y_bf16 == x_bf16) return MOE_ERR_INVALID_ARG;
@@ -247,7 +249,7 @@ moe_status moe_expert_ffn_prefill(const moe_layer* layer, const void* x_bf16, in
   if (!topk_ids || !topk_w || !y_bf16) return MOE_ERR_INVALID_ARG;
   if (flags & ~(MOE_F_PRENORM | MOE_F_RESIDUAL | MOE_F_DETERMINISTIC | MOE_F_DEBUG))
     return MOE_ERR_INVALID_ARG;
-  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, &L, &lay);
+  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, false, &L, &lay);
   if (s != MOE_OK) return s;
   if (!aligned16(y_bf16)) return MOE_ERR_MISALIGNED;
   if (y_bf16 == x_bf16) return MOE_ERR_INVALID_ARG;
@@ -264,7 +266,7 @@ moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t
   LayerDev L;
   WsLayout lay;
   if (!y_bf16) return MOE_ERR_INVALID_ARG;
-  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, &L, &lay);
+  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, T <= 4, &L, &lay);
   if (s != MOE_OK) return s;
   if (y_bf16 == x_bf16) return MOE_ERR_INVALID_ARG;
   if (flags & ~(MOE_F_PRENORM | MOE_F_RESIDUAL | MOE_F_DETERMINISTIC | MOE_F_DEBUG))

@@ -82,10 +82,11 @@ struct PfWs {
 
 // Internal positions: every bucket starts at a multiple of PF_PAD rows (so that
 // whole 32-row blocks of a chunk stay inside its bucket); the padding rows
-// carry token -1.
+// carry token -1.  At most min(E, T*k) + 1 buckets are non-empty.
 constexpr int PF_PAD = 32;
 static size_t pf_rows(const LayerDev& L, int T) {
-  return (size_t)T * (L.k + 1) + (size_t)PF_PAD * (L.E + 1);
+  const size_t nonempty = (size_t)((long long)T * L.k < L.E ? (long long)T * L.k : L.E) + 1;
+  return (size_t)T * (L.k + 1) + (size_t)PF_PAD * nonempty;
 }
 
 static size_t pf_max_chunks(const LayerDev& L, int T) {
