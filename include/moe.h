@@ -108,7 +108,7 @@ typedef struct {
 
 /* Bytes of workspace the calls below need for up to max_tokens tokens
  * (0 on invalid arguments).  The decode path (moe_route_topk with T <= 8,
- * moe_expert_ffn_decode, moe_block_forward with T <= 4) uses only a leading
+ * moe_expert_ffn_decode, moe_block_forward with T <= 8) uses only a leading
  * part of the layout and accepts any workspace at least that large; the
  * prefill path needs the full size. */
 size_t moe_workspace_bytes(const moe_layer* layer, int32_t max_tokens);
@@ -152,8 +152,9 @@ moe_status moe_expert_ffn_prefill(const moe_layer* layer, const void* x_bf16, in
                                   int32_t* bucket_offsets_or_null, int32_t* bucket_entries_or_null,
                                   uint32_t flags, void* ws, size_t ws_bytes, void* stream);
 
-/* The whole block: moe_route_topk, then the decode step for T <= 4 and the
- * prefill step otherwise.  Routing lists live in the workspace. */
+/* The whole block: moe_route_topk, then the decode step for T <= 8 (faster
+ * than the prefill step at every window it supports) and the prefill step
+ * otherwise.  Routing lists live in the workspace. */
 moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t T, void* y_bf16,
                              uint32_t flags, void* ws, size_t ws_bytes, void* stream);
 

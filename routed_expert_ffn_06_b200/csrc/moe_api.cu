@@ -266,7 +266,7 @@ moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t
   LayerDev L;
   WsLayout lay;
   if (!y_bf16) return MOE_ERR_INVALID_ARG;
-  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, T <= 4, &L, &lay);
+  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, T <= kMaxDecodeT, &L, &lay);
   if (s != MOE_OK) return s;
   if (y_bf16 == x_bf16) return MOE_ERR_INVALID_ARG;
   if (flags & ~(MOE_F_PRENORM | MOE_F_RESIDUAL | MOE_F_DETERMINISTIC | MOE_F_DEBUG))
@@ -279,7 +279,7 @@ moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t
   float* wt = reinterpret_cast<float*>(w + lay.w);
   s = moe_route_topk(layer, x_bf16, T, flags, nullptr, ids, wt, ws, ws_bytes, stream);
   if (s != MOE_OK) return s;
-  if (T <= 4)
+  if (T <= kMaxDecodeT)   // the decode kernels are faster up to their 8-token limit
     return moe_expert_ffn_decode(layer, x_bf16, T, ids, wt, y_bf16, flags, ws, ws_bytes, stream);
   return moe_expert_ffn_prefill(layer, x_bf16, T, ids, wt, y_bf16, nullptr, nullptr, flags, ws,
                                 ws_bytes, stream);

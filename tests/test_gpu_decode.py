@@ -164,3 +164,19 @@ def test_decode_wide_model(T):
     y = gb.decode(x, ids, w)
     oracle_check(layer, x, logits, ids, w, y)
     assert gb.error_word() == (0, 0)
+
+
+@pytest.mark.parametrize("T", [5, 8])
+def test_block_forward_uses_decode_up_to_eight_tokens(T):
+    """moe_block_forward on a 5- and an 8-token window (decode path): routing
+    and outputs match the oracle, and equal the expert step called directly."""
+    wl = synth.WORKLOADS["decode"]
+    layer = synth.make_layer(wl["shape"], seed=6, device="cuda", bias=wl["bias"], slot=wl["slot"])
+    x = synth.make_tokens(T, 2048, seed=30 + T, device="cuda")
+    gb = GpuBlock(layer, T)
+    logits, ids, w = gb.route(x)
+    y = gb.block(x)
+    yd = gb.decode(x, ids, w)
+    torch.cuda.synchronize()
+    assert torch.equal(y, yd)
+    oracle_check(layer, x, logits, ids, w, y)
