@@ -719,9 +719,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
     KSeq q;
     q.init(a, n_items);
     if (grp == 1 && !q.done) q.advance(a);
-    // Two register buffers alternate: the codes of the group's next k-step
-    // load while the current one is dequantised, and no copy of a buffer
-    // waits on its loads.
+    // Rotating register buffers: no copy of a buffer ever waits on its loads.
     auto produce = [&](const PfRaw& r, int g) {
       const int sa = g % PF_NS;
       if (g >= PF_NS && ok) ok = mbar_wait(&empty[sa], ((g / PF_NS) - 1) & 1, ctl, 0x611);
@@ -752,30 +750,47 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
       q.advance(a);
       if (!q.done) q.advance(a);
     };
-    PfRaw r0, r1;
+    PfRaw r0, r1, r2;
     PfUnits U;
     U.key = -1;
-    bool have0 = !q.done;
-    if (have0) {
+    // three buffers: the codes of the group's next two k-steps are in flight
+    // while the current one is dequantised
+    bool h0 = false, h1 = false, h2 = false;
+    if (!q.done) {
       pf_load_raw<BITS>(a, q, rq, gi, U, r0);
       skip2();
+      h0 = true;
+    }
+    if (!q.done) {
+      pf_load_raw<BITS>(a, q, rq, gi, U, r1);
+      skip2();
+      h1 = true;
     }
     int g = grp;
-    while (have0) {
-      const bool have1 = !q.done;
-      if (have1) {
-        pf_load_raw<BITS>(a, q, rq, gi, U, r1);
+    for (;;) {
+      if (!h0) break;
+      h2 = !q.done;
+      if (h2) {
+        pf_load_raw<BITS>(a, q, rq, gi, U, r2);
         skip2();
       }
       produce(r0, g);
       g += 2;
-      if (!have1) break;
-      have0 = !q.done;
-      if (have0) {
+      if (!h1) break;
+      h0 = !q.done;
+      if (h0) {
         pf_load_raw<BITS>(a, q, rq, gi, U, r0);
         skip2();
       }
       produce(r1, g);
+      g += 2;
+      if (!h2) break;
+      h1 = !q.done;
+      if (h1) {
+        pf_load_raw<BITS>(a, q, rq, gi, U, r1);
+        skip2();
+      }
+      produce(r2, g);
       g += 2;
     }
   } else if (warp == 13) {
