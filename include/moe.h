@@ -108,9 +108,9 @@ typedef struct {
 
 /* Bytes of workspace the calls below need for up to max_tokens tokens
  * (0 on invalid arguments).  The decode path (moe_route_topk with T <= 8,
- * moe_expert_ffn_decode, moe_block_forward with T <= 8) uses only a leading
- * part of the layout and accepts any workspace at least that large; the
- * prefill path needs the full size. */
+ * moe_expert_ffn_decode, moe_block_forward with T <= 8 on a layer the decode
+ * kernels take) uses only a leading part of the layout and accepts any
+ * workspace at least that large; the prefill path needs the full size. */
 size_t moe_workspace_bytes(const moe_layer* layer, int32_t max_tokens);
 
 /* Zero a workspace (enqueued on stream).  Needed once after allocation. */
@@ -134,7 +134,13 @@ moe_status moe_route_topk(const moe_layer* layer, const void* x_bf16, int32_t T,
  * experts (deduplicated across the window) and the shared expert, combined
  * with the routing weights.  Weight bytes are streamed once per call.
  *  topk_ids/topk_w: dev, as written by moe_route_topk.  y_bf16: dev bf16 [T][d]
- *  (may not alias x).  flags: PRENORM, RESIDUAL, DEBUG. */
+ *  (may not alias x).  flags: PRENORM, RESIDUAL, DEBUG.
+ *  Returns MOE_ERR_UNSUPPORTED_SHAPE, before enqueuing anything, for T > 8 and
+ *  for experts too wide for the kernels' shared-memory stages: each of 16
+ *  warps stages one expert's whole down-projection tile with its hidden
+ *  vectors, so the limit on max(ffn, shared_ffn) falls as T grows (d 2048 and
+ *  512 experts: up to 1888 (2-bit) / 1472 (3-bit) at T = 1, 608 / 576 at
+ *  T = 8). */
 moe_status moe_expert_ffn_decode(const moe_layer* layer, const void* x_bf16, int32_t T,
                                  const int32_t* topk_ids, const float* topk_w, void* y_bf16,
                                  uint32_t flags, void* ws, size_t ws_bytes, void* stream);
@@ -152,9 +158,10 @@ moe_status moe_expert_ffn_prefill(const moe_layer* layer, const void* x_bf16, in
                                   int32_t* bucket_offsets_or_null, int32_t* bucket_entries_or_null,
                                   uint32_t flags, void* ws, size_t ws_bytes, void* stream);
 
-/* The whole block: moe_route_topk, then the decode step for T <= 8 (faster
- * than the prefill step at every window it supports) and the prefill step
- * otherwise.  Routing lists live in the workspace. */
+/* The whole block: moe_route_topk, then the decode step for T <= 8 when the
+ * layer fits the decode kernels (faster than the prefill step at every window
+ * it supports) and the prefill step otherwise.  Routing lists live in the
+ * workspace. */
 moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t T, void* y_bf16,
                              uint32_t flags, void* ws, size_t ws_bytes, void* stream);
 
@@ -173,7 +180,9 @@ moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t
  *    stream, or events); overlapping calls race on the scratch.
  *  - Shapes whose workspace (moe_workspace_bytes(layer, T)) exceeds 2 MiB
  *    return MOE_ERR_WORKSPACE_TOO_SMALL; T > 4 returns
- *    MOE_ERR_UNSUPPORTED_SHAPE; both before anything is enqueued.
+ *    MOE_ERR_UNSUPPORTED_SHAPE; both before anything is enqueued.  A layer
+ *    too wide for the decode kernels (see moe_expert_ffn_decode) takes the
+ *    prefill step, whose full workspace must then fit in the 2 MiB.
  *  - Device-side error bits go to the array's control block, which no entry
  *    point reads back; use moe_block_forward with a workspace to inspect them. */
 moe_status moe_block_forward_noalloc(const moe_layer* layer, const void* x_bf16, int32_t T,

@@ -680,6 +680,21 @@ __global__ void __launch_bounds__(kDnWarps * 32, 1)
 constexpr size_t kGuSmemBudget = 215 * 1024;
 constexpr size_t kDnSmemBudget = 215 * 1024;
 
+// The stage counts above aim at the budgets; with one stage per warp a launch
+// may go up to the sm_100 opt-in maximum of shared memory per block (232448
+// bytes), less a margin for the kernels' static shared variables.
+constexpr size_t kSmemPerBlockMax = 232448 - 256;
+
+// Whether a T-token window of this layer fits the decode kernels: one stage per
+// warp must hold a whole expert's Wd tile and hidden vectors (16 warps), and
+// the gate/up kernel its token copies.  Wider experts take the prefill path.
+bool decode_fits(int d, int E, int Fmax, int bits, int T) {
+  if (d <= 0 || E <= 0 || Fmax <= 0 || T < 1 || T > kMaxDecodeT || (bits != 2 && bits != 3))
+    return false;
+  return gu_smem(d, E, bits, 1).total <= kSmemPerBlockMax &&
+         dn_smem(E, bits, Fmax, T, 1).total <= kSmemPerBlockMax;
+}
+
 template <int BITS>
 static cudaError_t launch_decode_bits(const LayerDev& L, const uint16_t* x, int T,
                                       const int32_t* ids, const float* w, uint16_t* y,

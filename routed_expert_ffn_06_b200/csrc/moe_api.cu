@@ -231,6 +231,8 @@ moe_status moe_expert_ffn_decode(const moe_layer* layer, const void* x_bf16, int
   if (T > kMaxDecodeT) return MOE_ERR_UNSUPPORTED_SHAPE;
   moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, true, &L, &lay);
   if (s != MOE_OK) return s;
+  if (T > 0 && !decode_fits(L.d, L.E, L.F > L.Fs ? L.F : L.Fs, L.bits, T))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(y_bf16)) return MOE_ERR_MISALIGNED;
   if (y_bf16 == x_bf16) return MOE_ERR_INVALID_ARG;
   if ((s = check_device()) != MOE_OK) return s;
@@ -265,8 +267,13 @@ moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t
                              uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
   LayerDev L;
   WsLayout lay;
-  if (!y_bf16) return MOE_ERR_INVALID_ARG;
-  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, T <= kMaxDecodeT, &L, &lay);
+  if (!y_bf16 || !layer) return MOE_ERR_INVALID_ARG;
+  // the decode kernels are faster up to their 8-token limit, for layers whose
+  // experts fit their shared-memory stages
+  const int Fmax = layer->ffn > layer->shared_ffn ? layer->ffn : layer->shared_ffn;
+  const bool dec = T <= kMaxDecodeT &&
+                   (T == 0 || decode_fits(layer->d_model, layer->n_experts, Fmax, layer->bits, T));
+  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, dec, &L, &lay);
   if (s != MOE_OK) return s;
   if (y_bf16 == x_bf16) return MOE_ERR_INVALID_ARG;
   if (flags & ~(MOE_F_PRENORM | MOE_F_RESIDUAL | MOE_F_DETERMINISTIC | MOE_F_DEBUG))
@@ -279,7 +286,7 @@ moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t
   float* wt = reinterpret_cast<float*>(w + lay.w);
   s = moe_route_topk(layer, x_bf16, T, flags, nullptr, ids, wt, ws, ws_bytes, stream);
   if (s != MOE_OK) return s;
-  if (T <= kMaxDecodeT)   // the decode kernels are faster up to their 8-token limit
+  if (dec)
     return moe_expert_ffn_decode(layer, x_bf16, T, ids, wt, y_bf16, flags, ws, ws_bytes, stream);
   return moe_expert_ffn_prefill(layer, x_bf16, T, ids, wt, y_bf16, nullptr, nullptr, flags, ws,
                                 ws_bytes, stream);

@@ -102,8 +102,20 @@ def oracle_check(layer, x, logits, ids, w, y, flags=0, rows=None, oflags=None):
         xin = x.cpu().double().numpy()[rr]
     bound = logit_bound(layer, xin)
     assert np.all(np.abs(lg[rr] - r["logits"]) <= bound), "router logits outside the fp32 bound"
+    # The weights are the softmax of the selected logits, which the device
+    # knows to fp32 accuracy only: (a) against the softmax, in fp64, of the
+    # device's own selected logits (the weight arithmetic alone), tightly; (b)
+    # against the oracle's weights within the propagated logit error,
+    # |dw_j| <= w_j * expm1(2 max_i |dl_i|) over the selected i.
     wg = w.cpu().double().numpy()[rr]
-    assert np.allclose(wg, r["w"], rtol=1e-5, atol=1e-6), "routing weights differ"
+    sel = np.take_along_axis(lg[rr].astype(np.float64), ids_g.astype(np.int64), axis=1)
+    own = np.exp(sel - sel.max(1, keepdims=True))
+    own /= own.sum(1, keepdims=True)
+    assert np.allclose(wg, own, rtol=1e-5, atol=1e-6), "weights differ from the softmax of the logits"
+    dl = np.take_along_axis(np.abs(lg[rr].astype(np.float64) - r["logits"]),
+                            ids_g.astype(np.int64), axis=1).max(1, keepdims=True)
+    assert np.all(np.abs(wg - r["w"]) <= r["w"] * (np.expm1(2 * dl) + 1e-5) + 1e-6), \
+        "routing weights outside the logit-error bound"
     assert np.allclose(wg.sum(1), 1.0, atol=1e-6)
     yg = y.float().cpu().double().numpy()[rr]
     return assert_close(yg, r["y"])

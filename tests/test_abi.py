@@ -108,3 +108,16 @@ def test_status_strings(lib):
     assert moe.moe_status_string(0) == "ok"
     assert "workspace" in moe.moe_status_string(3)
     assert "sm_100a" in moe.moe_build_info()
+
+
+def test_decode_rejects_experts_too_wide_for_its_stages(lib):
+    """The decode step checks that its shared-memory stages hold the layer
+    before anything else touches the device: ffn 4096 at d 256 is a valid layer
+    that only the prefill step takes (MOE_ERR_UNSUPPORTED_SHAPE, not a launch
+    failure), while ffn 512 passes the shape checks and stops at the missing
+    device."""
+    x, y, ids, w, ws = 0x7F0000400000, 0x7F0000500000, 0x7F0000700000, 0x7F0000800000, 0x7F0000600000
+    wide = _layer(d_model=256, n_experts=20, ffn=4096, shared_ffn=4096, top_k=16)
+    assert lib.moe_expert_ffn_decode(ctypes.byref(wide), x, 1, ids, w, y, 0, ws, 1 << 30, None) == 2
+    ok = _layer(d_model=256, n_experts=20, ffn=512, shared_ffn=512, top_k=16)
+    assert lib.moe_expert_ffn_decode(ctypes.byref(ok), x, 8, ids, w, y, 0, ws, 1 << 30, None) == 8

@@ -205,3 +205,58 @@ def test_router_large_T_tensor_core(T, d, E):
     assert np.array_equal(oracle.select_topk_f32(lg, sh.k), ids.cpu().numpy())
     assert np.allclose(w.sum(1).cpu().numpy(), 1.0, atol=1e-5)
     assert gb.error_word() == (0, 0)
+
+
+def test_prefill_hot_experts_split_into_many_chunks():
+    """Every token routes to the same k experts (router bias far above the
+    token logits), so k buckets hold all T tokens, several 128-token chunks
+    each, and every other routed bucket is empty."""
+    sh = synth.MoEShape(d=128, E=32, F=64, Fs=64, k=4, bits=3)
+    layer = synth.make_layer(sh, seed=7, device="cuda", bias="normal")
+    hot = [3, 11, 20, 31]
+    b = torch.zeros(sh.E, dtype=torch.float32)
+    b[hot] = torch.tensor([12.0, 11.5, 11.0, 10.5])
+    layer.router_bias.copy_(b.to("cuda"))
+    T = 600
+    x = synth.make_tokens(T, sh.d, seed=8, device="cuda")
+    gb = GpuBlock(layer, T)
+    logits, ids, w = gb.route(x)
+    assert sorted(ids.unique().tolist()) == hot
+    y, off, ent = gb.prefill(x, ids, w, want_buckets=True)
+    _check_buckets(ids, off, ent, sh.E)
+    counts = np.diff(off.cpu().numpy())[:sh.E]
+    assert counts[hot].tolist() == [T] * 4 and int(counts.sum()) == 4 * T
+    oracle_check(layer, x, logits, ids, w, y)
+    assert gb.error_word() == (0, 0)
+
+
+def test_prefill_zero_tokens_is_a_noop():
+    sh = synth.MoEShape(d=128, E=32, F=64, Fs=64, k=4, bits=2)
+    layer = synth.make_layer(sh, seed=1, device="cuda", bias="normal")
+    gb = GpuBlock(layer, 16)
+    x = torch.ones(1, 128, dtype=torch.bfloat16, device="cuda")
+    ids = torch.zeros(1, 4, dtype=torch.int32, device="cuda")
+    w = torch.zeros(1, 4, dtype=torch.float32, device="cuda")
+    y = torch.full((1, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_ffn_prefill(gb.L, x, 0, ids, w, y, None, None, 0, gb.ws)
+    torch.cuda.synchronize()
+    assert torch.all(y == 7.0)
+    assert gb.error_word() == (0, 0)
+
+
+@pytest.mark.parametrize("d,F,T,n_rows", [(4096, 1024, 40, 8), (256, 4096, 300, 20)])
+def test_prefill_widest_shapes(d, F, T, n_rows):
+    """The largest supported model width (4096) or expert width (4096) with
+    the largest top-k (16), 3-bit: buckets exact, and routing and outputs
+    against the oracle on the first and last token and a seeded sample."""
+    sh = synth.MoEShape(d=d, E=20, F=F, Fs=F, k=16, bits=3)
+    layer = synth.make_layer(sh, seed=13, device="cuda", bias="normal")
+    x = synth.make_tokens(T, d, seed=14, device="cuda")
+    gb = GpuBlock(layer, T)
+    logits, ids, w = gb.route(x)
+    y, off, ent = gb.prefill(x, ids, w, want_buckets=True)
+    _check_buckets(ids, off, ent, sh.E)
+    rng = np.random.default_rng(T)
+    rows = np.unique(np.concatenate([[0, T - 1], rng.choice(T, n_rows - 2, replace=False)]))
+    oracle_check(layer, x, logits, ids, w, y, rows=rows)
+    assert gb.error_word() == (0, 0)
