@@ -40,7 +40,7 @@ def test_tiny_config_block():
 
 @pytest.mark.parametrize("bits", [2, 3])
 @pytest.mark.parametrize("T", [1, 2, 3, 5, 8])
-@pytest.mark.parametrize("E,k,Fs", [(16, 2, 32), (37, 5, 0), (64, 16, 64), (8, 8, 32)])
+@pytest.mark.parametrize("E,k,Fs", [(16, 2, 32), (37, 5, 0), (64, 16, 64), (8, 8, 32), (12, 1, 32)])
 def test_small_shapes(bits, T, E, k, Fs):
     sh = synth.MoEShape(d=96, E=E, F=64, Fs=Fs, k=k, bits=bits)
     layer = _layer(sh, seed=T * 7 + E, bias_std=1.0)

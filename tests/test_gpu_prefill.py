@@ -42,7 +42,9 @@ def test_tiny_config_prefill(T):
 @pytest.mark.parametrize("shape", [dict(d=128, E=32, F=64, Fs=64, k=4),
                                    dict(d=256, E=64, F=128, Fs=0, k=6),
                                    dict(d=192, E=40, F=96, Fs=160, k=3),
-                                   dict(d=160, E=24, F=64, Fs=32, k=2)])
+                                   dict(d=160, E=24, F=64, Fs=32, k=2),
+                                   dict(d=128, E=16, F=64, Fs=0, k=1),
+                                   dict(d=96, E=6, F=64, Fs=32, k=6)])
 def test_prefill_small_shapes(bits, shape):
     sh = synth.MoEShape(bits=bits, **shape)
     layer = synth.make_layer(sh, seed=11, device="cuda", bias="normal", bias_std=1.0)
