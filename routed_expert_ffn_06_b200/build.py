@@ -17,8 +17,11 @@ NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", 
               "-Xptxas", "-warn-spills"]
 
 
+HOST = os.path.join(PKG, "host")   # host-only code (the weight packer)
+
+
 def sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu"))) + sorted(glob.glob(os.path.join(HOST, "*.cu")))
 
 
 def stale() -> bool:
@@ -26,7 +29,7 @@ def stale() -> bool:
         return True
     t = os.path.getmtime(LIB)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
-    deps += [os.path.join(INCLUDE, "moe.h")]
+    deps += glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(p) > t for p in deps)
 
 

@@ -31,7 +31,7 @@ F_DEBUG = 8
 
 EXPORTS = ["moe_workspace_bytes", "moe_workspace_init", "moe_workspace_error", "moe_route_topk",
            "moe_expert_ffn_decode", "moe_expert_ffn_prefill", "moe_block_forward",
-           "moe_block_forward_noalloc", "moe_status_string", "moe_build_info"]
+           "moe_block_forward_noalloc", "moe_status_string", "moe_build_info", "moe_pack_host"]
 
 
 class MoEError(RuntimeError):
@@ -85,6 +85,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.moe_status_string.argtypes = [st]
     L.moe_build_info.restype = ctypes.c_char_p
     L.moe_build_info.argtypes = []
+    L.moe_pack_host.restype = st
+    L.moe_pack_host.argtypes = [vp, i32, i32, i32, vp, vp]
     _lib = L
     return L
 
@@ -177,6 +179,23 @@ def moe_block_forward_noalloc(layer: moe_layer, x, T: int, y, flags: int, stream
     _check(load().moe_block_forward_noalloc(ctypes.byref(layer), _ptr(x), int(T), _ptr(y),
                                             int(flags), _stream(stream)),
            "moe_block_forward_noalloc")
+
+
+def moe_pack_host(w, bits: int):
+    """Quantise and pack one host fp32 matrix [rows, cols] (include/moe_pack.h).
+    Returns (codes uint8 [rows/16, cols/32*16*(8|12)], scales int16 holding
+    fp16 bits [rows/16, cols/32*16]), host tensors."""
+    import torch
+    if w.device.type != "cpu" or w.dtype != torch.float32 or w.dim() != 2:
+        raise ValueError("moe_pack_host takes a 2-D host float32 tensor")
+    w = w.contiguous()
+    rows, cols = w.shape
+    gb = 8 if bits == 2 else 12
+    codes = torch.empty(max(rows // 16, 1), max(cols // 32, 1) * 16 * gb, dtype=torch.uint8)
+    scales = torch.empty(max(rows // 16, 1), max(cols // 32, 1) * 16, dtype=torch.int16)
+    _check(load().moe_pack_host(w.data_ptr(), int(rows), int(cols), int(bits), codes.data_ptr(),
+                                scales.data_ptr()), "moe_pack_host")
+    return codes, scales
 
 
 def moe_status_string(status: int) -> str:
