@@ -80,6 +80,42 @@ class GpuBlock:
         return moe.moe_workspace_error(self.ws)
 
 
+def router_oracle(layer):
+    """The oracle for one layer's router only: host copies of the router
+    tensors (its router reads no expert bytes, so those stay where they are)."""
+    z8 = torch.zeros(16, dtype=torch.uint8)
+    z16 = torch.zeros(16, dtype=torch.float16)
+    lite = synth.Layer(layer.shape, layer.router_w.cpu(), None if layer.router_bias is None
+                       else layer.router_bias.cpu(), layer.expert_slot.cpu(), z8, z16, None, None)
+    return oracle.OracleLayer(lite)
+
+
+def routing_check(layer, x, logits, ids, w, flags=0):
+    """Routing of every token of one layer against the oracle: selection on
+    the device's fp32 logits, logits within the fp32 bound of the oracle's
+    fp64 router, weights as in oracle_check."""
+    lg = logits.cpu().numpy()
+    ids_g = ids.cpu().numpy()
+    assert np.array_equal(oracle.select_topk_f32(lg, layer.shape.k), ids_g), "routing differs"
+    if flags & moe.F_PRENORM:
+        xin = oracle.rmsnorm_bf16(bf16_bits(x))
+        xin = torch.from_numpy(xin.view(np.int16)).view(torch.bfloat16).double().numpy()
+    else:
+        xin = x.cpu().double().numpy()
+    lg64 = router_oracle(layer).router_logits(xin)
+    assert np.all(np.abs(lg - lg64) <= logit_bound(layer, xin)), "router logits outside the fp32 bound"
+    wg = w.cpu().double().numpy()
+    sel = np.take_along_axis(lg.astype(np.float64), ids_g.astype(np.int64), axis=1)
+    own = np.exp(sel - sel.max(1, keepdims=True))
+    own /= own.sum(1, keepdims=True)
+    assert np.allclose(wg, own, rtol=1e-5, atol=1e-6), "weights differ from the softmax of the logits"
+    ref = oracle.renorm_weights(lg64, ids_g)
+    dl = np.take_along_axis(np.abs(lg.astype(np.float64) - lg64), ids_g.astype(np.int64),
+                            axis=1).max(1, keepdims=True)
+    assert np.all(np.abs(wg - ref) <= ref * (np.expm1(2 * dl) + 1e-5) + 1e-6), \
+        "routing weights outside the logit-error bound"
+
+
 def oracle_check(layer, x, logits, ids, w, y, flags=0, rows=None, oflags=None):
     """Compare one GPU block result with the oracle (selection on the GPU's
     fp32 logits).  Returns (max rel, rms rel)."""

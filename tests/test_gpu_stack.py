@@ -8,7 +8,7 @@ import pytest
 import torch
 
 from routed_expert_ffn_06_b200 import build, moe, synth
-from _util import GpuBlock, oracle_check
+from _util import GpuBlock, oracle_check, routing_check
 
 pytestmark = pytest.mark.gpu
 
@@ -61,3 +61,32 @@ def test_mix_prefill_then_decode_with_drift():
     for layer in layers:
         layer.router_bias.copy_(synth.permute_profile(layer, seed=0, epoch=1))
     _run_layers(layers, win)
+
+
+def test_decode_stack_all_48_layers():
+    """The whole 48-layer 3-bit decode stack, one 4-token step through
+    moe_block_forward with pre-norm and residual, teacher-forced.  At every
+    layer the routing of every token is checked against the oracle (selection
+    on the device's fp32 logits, logits within the fp32 bound of the oracle's
+    fp64 router, weights); at the first, a middle and the last layer the
+    outputs too.  Layers are generated one at a time, so the stack's 34 GB never
+    sit on the device together."""
+    wl = synth.WORKLOADS["decode_stack"]
+    sh = wl["shape"]
+    T = 4
+    x = synth.make_tokens(T, sh.d, seed=77, device="cuda")
+    for l in range(48):
+        layer = synth.make_layer(sh, seed=0, layer=l, device="cuda", bias=wl["bias"],
+                                 slot=wl["slot"])
+        gb = GpuBlock(layer, T)
+        logits, ids, w = gb.route(x, FLAGS)
+        y = gb.block(x, FLAGS)
+        torch.cuda.synchronize()
+        if l in (0, 24, 47):
+            oracle_check(layer, x, logits, ids, w, y, flags=FLAGS)
+        else:
+            routing_check(layer, x, logits, ids, w, flags=FLAGS)
+        assert gb.error_word() == (0, 0)
+        assert torch.isfinite(y.float()).all()
+        x = y
+        del layer, gb
