@@ -7,6 +7,8 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
+
 from routed_expert_ffn_06_b200 import build, moe, synth
 from _util import GpuBlock, oracle_check, routing_check
 
@@ -88,5 +90,33 @@ def test_decode_stack_all_48_layers():
             routing_check(layer, x, logits, ids, w, flags=FLAGS)
         assert gb.error_word() == (0, 0)
         assert torch.isfinite(y.float()).all()
+        x = y
+        del layer, gb
+
+
+def test_mix_prefill_chunk_all_48_layers():
+    """One full 8192-token chunk of the mix through all 48 3-bit layers with
+    pre-norm and residual, teacher-forced.  At every layer the selection of
+    every token equals the oracle's on the device's fp32 logits; at the first,
+    a middle and the last layer a seeded sample of 24 tokens is checked in full
+    (logits, weights, outputs) against the oracle."""
+    wl = synth.WORKLOADS["mix"]
+    sh = wl["shape"]
+    T = wl["chunk"]
+    x = synth.make_tokens(T, sh.d, seed=5, device="cuda")
+    rows = np.unique(np.random.default_rng(5).choice(T, 24, replace=False))
+    for l in range(48):
+        layer = synth.make_layer(sh, seed=0, layer=l, device="cuda", bias=wl["bias"],
+                                 slot=wl["slot"])
+        gb = GpuBlock(layer, T)
+        logits, ids, w = gb.route(x, FLAGS)
+        y = gb.block(x, FLAGS)
+        torch.cuda.synchronize()
+        if l in (0, 24, 47):
+            oracle_check(layer, x, logits, ids, w, y, flags=FLAGS, rows=rows)
+        else:
+            assert np.array_equal(oracle.select_topk_f32(logits.cpu().numpy(), sh.k),
+                                  ids.cpu().numpy()), f"routing differs at layer {l}"
+        assert gb.error_word() == (0, 0)
         x = y
         del layer, gb
