@@ -125,3 +125,18 @@ def test_decode_rejects_experts_too_wide_for_its_stages(lib):
     assert lib.moe_expert_ffn_decode(ctypes.byref(wide), x, 1, ids, w, y, 0, ws, 1 << 30, None) == 2
     ok = _layer(d_model=256, n_experts=20, ffn=512, shared_ffn=512, top_k=16)
     assert lib.moe_expert_ffn_decode(ctypes.byref(ok), x, 8, ids, w, y, 0, ws, 1 << 30, None) == 8
+
+
+def test_block_forward_takes_prefill_for_experts_too_wide_for_decode(lib):
+    """Path choice on the host, seen through the workspace it demands: a
+    4-token window of a layer within the decode kernels' width runs the decode
+    path, which needs only a leading part of the workspace (so one byte short
+    of the full size passes and the call stops at the missing device); with
+    ffn 4096 the same window takes the prefill path, which needs it all."""
+    x, y = 0x7F0000400000, 0x7F0000500000
+    for ffn, want in [(512, 8), (4096, 3)]:
+        L = _layer(d_model=256, n_experts=20, ffn=ffn, shared_ffn=ffn, top_k=16)
+        full = lib.moe_workspace_bytes(ctypes.byref(L), 4)
+        assert full > 0
+        rc = lib.moe_block_forward(ctypes.byref(L), x, 4, y, 0, 0x7F0000600000, full - 1, None)
+        assert rc == want, (ffn, rc)
