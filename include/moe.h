@@ -173,18 +173,23 @@ moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t
  * device).
  *  - Allocates nothing.  The first call on a device (with that device
  *    current) looks up the array's address with cudaGetSymbolAddress; make
- *    that first call before any stream capture.
- *  - The array starts zeroed (module load) and every call leaves its control
- *    block zeroed again; nothing else has to be initialised.
+ *    that first call before any stream capture.  The address is cached with
+ *    the id of the CUDA context it came from and looked up again when the
+ *    current context changes (after a device reset, for instance).
+ *  - Every call that passes validation first zeroes the array's 256-byte
+ *    control block with an enqueued cudaMemsetAsync (error word, counters);
+ *    nothing else has to be initialised.  Device-side error bits cannot be
+ *    read back through this entry point; use moe_block_forward with a
+ *    workspace to inspect them.
  *  - One scratch per device: calls on the same device must be ordered (one
- *    stream, or events); overlapping calls race on the scratch.
+ *    stream, or events); calls that overlap on the GPU race on the scratch.
  *  - Shapes whose workspace (moe_workspace_bytes(layer, T)) exceeds 2 MiB
  *    return MOE_ERR_WORKSPACE_TOO_SMALL; T > 4 returns
  *    MOE_ERR_UNSUPPORTED_SHAPE; both before anything is enqueued.  A layer
  *    too wide for the decode kernels (see moe_expert_ffn_decode) takes the
  *    prefill step, whose full workspace must then fit in the 2 MiB.
- *  - Device-side error bits go to the array's control block, which no entry
- *    point reads back; use moe_block_forward with a workspace to inspect them. */
+ *  - Status codes match moe_block_forward's (MOE_ERR_NO_DEVICE without a
+ *    current sm_100 device). */
 moe_status moe_block_forward_noalloc(const moe_layer* layer, const void* x_bf16, int32_t T,
                                      void* y_bf16, uint32_t flags, void* stream);
 

@@ -88,4 +88,14 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 int sm_count();
 
+// MOE_OK when the current device is an sm_100 GPU (cached per device), else
+// MOE_ERR_NO_DEVICE.
+moe_status check_device();
+
+// moe_block_forward with an option to zero the workspace control block on the
+// stream (after validation, before the first kernel).
+moe_status block_forward(const moe_layer* layer, const void* x_bf16, int32_t T, void* y_bf16,
+                         uint32_t flags, void* ws, size_t ws_bytes, void* stream,
+                         bool clear_control);
+
 }  // namespace moe

@@ -24,6 +24,8 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
 moe_status check_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -42,6 +44,8 @@ moe_status check_device() {
   }
   return g_dev_ok[dev] == 1 ? MOE_OK : MOE_ERR_NO_DEVICE;
 }
+
+namespace {
 
 moe_status validate_layer(const moe_layer* l) {
   if (!l) return MOE_ERR_INVALID_ARG;
@@ -156,6 +160,44 @@ WsLayout ws_layout(const LayerDev& L, int T) {
   return w;
 }
 
+
+// The block forward behind moe_block_forward (and the allocation-free entry
+// point): every argument is validated first; with clear_control the
+// workspace's control block is zeroed on the stream just before the kernels.
+moe_status block_forward(const moe_layer* layer, const void* x_bf16, int32_t T, void* y_bf16,
+                         uint32_t flags, void* ws, size_t ws_bytes, void* stream,
+                         bool clear_control) {
+  LayerDev L;
+  WsLayout lay;
+  if (!y_bf16 || !layer) return MOE_ERR_INVALID_ARG;
+  // the decode kernels are faster up to their 8-token limit, for layers whose
+  // experts fit their shared-memory stages
+  const int Fmax = layer->ffn > layer->shared_ffn ? layer->ffn : layer->shared_ffn;
+  const bool dec = T <= kMaxDecodeT &&
+                   (T == 0 || decode_fits(layer->d_model, layer->n_experts, Fmax, layer->bits, T));
+  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, dec, &L, &lay);
+  if (s != MOE_OK) return s;
+  if (y_bf16 == x_bf16) return MOE_ERR_INVALID_ARG;
+  if (flags & ~(MOE_F_PRENORM | MOE_F_RESIDUAL | MOE_F_DETERMINISTIC | MOE_F_DEBUG))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_bf16)) return MOE_ERR_MISALIGNED;
+  if ((s = check_device()) != MOE_OK) return s;
+  if (T == 0) return MOE_OK;
+  char* w = static_cast<char*>(ws);
+  if (clear_control) {
+    s = from_cuda(cudaMemsetAsync(w + lay.ctl, 0, sizeof(Control), static_cast<cudaStream_t>(stream)));
+    if (s != MOE_OK) return s;
+  }
+  int32_t* ids = reinterpret_cast<int32_t*>(w + lay.ids);
+  float* wt = reinterpret_cast<float*>(w + lay.w);
+  s = moe_route_topk(layer, x_bf16, T, flags, nullptr, ids, wt, ws, ws_bytes, stream);
+  if (s != MOE_OK) return s;
+  if (dec)
+    return moe_expert_ffn_decode(layer, x_bf16, T, ids, wt, y_bf16, flags, ws, ws_bytes, stream);
+  return moe_expert_ffn_prefill(layer, x_bf16, T, ids, wt, y_bf16, nullptr, nullptr, flags, ws,
+                                ws_bytes, stream);
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -265,31 +307,7 @@ moe_status moe_expert_ffn_prefill(const moe_layer* layer, const void* x_bf16, in
 
 moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t T, void* y_bf16,
                              uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
-  LayerDev L;
-  WsLayout lay;
-  if (!y_bf16 || !layer) return MOE_ERR_INVALID_ARG;
-  // the decode kernels are faster up to their 8-token limit, for layers whose
-  // experts fit their shared-memory stages
-  const int Fmax = layer->ffn > layer->shared_ffn ? layer->ffn : layer->shared_ffn;
-  const bool dec = T <= kMaxDecodeT &&
-                   (T == 0 || decode_fits(layer->d_model, layer->n_experts, Fmax, layer->bits, T));
-  moe_status s = preamble(layer, T, x_bf16, ws, ws_bytes, dec, &L, &lay);
-  if (s != MOE_OK) return s;
-  if (y_bf16 == x_bf16) return MOE_ERR_INVALID_ARG;
-  if (flags & ~(MOE_F_PRENORM | MOE_F_RESIDUAL | MOE_F_DETERMINISTIC | MOE_F_DEBUG))
-    return MOE_ERR_INVALID_ARG;
-  if (!aligned16(y_bf16)) return MOE_ERR_MISALIGNED;
-  if ((s = check_device()) != MOE_OK) return s;
-  if (T == 0) return MOE_OK;
-  char* w = static_cast<char*>(ws);
-  int32_t* ids = reinterpret_cast<int32_t*>(w + lay.ids);
-  float* wt = reinterpret_cast<float*>(w + lay.w);
-  s = moe_route_topk(layer, x_bf16, T, flags, nullptr, ids, wt, ws, ws_bytes, stream);
-  if (s != MOE_OK) return s;
-  if (dec)
-    return moe_expert_ffn_decode(layer, x_bf16, T, ids, wt, y_bf16, flags, ws, ws_bytes, stream);
-  return moe_expert_ffn_prefill(layer, x_bf16, T, ids, wt, y_bf16, nullptr, nullptr, flags, ws,
-                                ws_bytes, stream);
+  return moe::block_forward(layer, x_bf16, T, y_bf16, flags, ws, ws_bytes, stream, false);
 }
 
 const char* moe_status_string(moe_status s) {

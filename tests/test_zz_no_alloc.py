@@ -1,14 +1,20 @@
 """moe_block_forward_noalloc: the decode-window block forward on the library's
-static device scratch, through the C ABI.  It must agree with the workspace
-entry point (moe_block_forward) on two calls in a row, and reject what its
-2 MiB scratch cannot hold before enqueuing anything."""
+static device scratch, for callers that cannot allocate device memory (a host
+with no device allocator, a step loop that must not call cudaMalloc because it
+synchronises the device).  Called through the C ABI, it must give exactly the
+bytes of the workspace entry point (moe_block_forward: same kernels, same
+inputs), on calls in a row and on calls queued back to back on one stream with
+no host synchronisation between them, and reject what its 2 MiB scratch cannot
+hold before enqueuing anything.
+
+This file sorts last so that a run stopping at its first failure has already
+run every other test."""
 import ctypes
 
 import pytest
 import torch
 
 from routed_expert_ffn_06_b200 import build, moe, synth
-from _util import assert_close
 
 pytestmark = pytest.mark.gpu
 
@@ -20,20 +26,25 @@ def _lib():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
 
 
+def _reference(L, x, T, flags):
+    """moe_block_forward on a workspace of its own."""
+    ws = moe.alloc_workspace(L, T)
+    y = torch.empty_like(x)
+    moe.moe_block_forward(L, x, T, y, flags, ws)
+    return y
+
+
 def _two_calls_match(layer, T, seed, flags=0):
     L = moe.make_layer_struct(layer)
-    ws = moe.alloc_workspace(L, T)
     x = synth.make_tokens(T, layer.shape.d, seed=seed, device="cuda")
     if flags & moe.F_PRENORM:
         x = (x.float() * 3).to(torch.bfloat16)
-    y_ref = torch.empty_like(x)
-    moe.moe_block_forward(L, x, T, y_ref, flags, ws)
+    y_ref = _reference(L, x, T, flags)
     for _ in range(2):
         y = torch.full_like(x, float("nan"))
         moe.moe_block_forward_noalloc(L, x, T, y, flags)
         torch.cuda.synchronize()
-        assert torch.isfinite(y.float()).all()
-        assert_close(y.float().cpu().double().numpy(), y_ref.float().cpu().double().numpy())
+        assert torch.equal(y, y_ref), "no-alloc output differs from the workspace entry point"
 
 
 @pytest.mark.parametrize("T", [1, 2, 3, 4])
@@ -54,6 +65,28 @@ def test_noalloc_tiny_config():
     wl = synth.WORKLOADS["tiny"]
     layer = synth.make_layer(wl["shape"], seed=0, device="cuda", bias=wl["bias"], slot=wl["slot"])
     _two_calls_match(layer, 4, seed=0)
+
+
+def test_noalloc_back_to_back_on_one_stream():
+    """Three calls with different inputs and separate outputs queued on one
+    stream with one synchronisation at the end: each must equal the workspace
+    entry point run on its own."""
+    wl = synth.WORKLOADS["decode"]
+    layers = [synth.make_layer(wl["shape"], seed=20 + i, device="cuda", bias=wl["bias"],
+                               slot=wl["slot"]) for i in range(2)]
+    Ls = [moe.make_layer_struct(l) for l in layers]
+    cases = [(0, 4, 100), (1, 1, 101), (0, 3, 102)]
+    xs = [synth.make_tokens(T, wl["shape"].d, seed=s, device="cuda") for _, T, s in cases]
+    refs = [_reference(Ls[li], x, T, 0) for (li, T, _), x in zip(cases, xs)]
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    ys = [torch.full_like(x, float("nan")) for x in xs]
+    with torch.cuda.stream(stream):
+        for (li, T, _), x, y in zip(cases, xs, ys):
+            moe.moe_block_forward_noalloc(Ls[li], x, T, y, 0, stream)
+    stream.synchronize()
+    for y, r in zip(ys, refs):
+        assert torch.equal(y, r), "queued no-alloc call differs from the workspace entry point"
 
 
 def _status(L, x, T, y):
