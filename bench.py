@@ -1,18 +1,21 @@
 """Benchmark of the routed sparse-MoE block on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|stack]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload decode|prefill|stack|mix] [--impl ours|reference]
 
-Default workload (the configuration the headline metric is quoted on): one
-routed-MoE layer, d=2048, 512 experts (SwiGLU ffn 512) + shared expert, top-10,
-2-bit group-32 weights with fp16 scales, Zipf(1.1) popularity, frequency-ordered
-slots; verify windows of T = 1, 2, 3 and 4 tokens.  A step is one pass of the
-block (router, top-k, expert FFNs, shared expert, combine) over each of the four
-windows, each on another of 32 independent layer copies (16 GB of weights, far
-above the 126 MB L2), with fresh tokens.  Steps are captured in a CUDA graph and
-replayed; the timed region is bracketed by a barrier and device syncs, timed with
-CUDA events, max over ranks.  One process per GPU; ranks run independent replicas
-(no collective on the data path).
+Default (the configuration the headline metric is quoted on): one routed-MoE
+layer, d=2048, 512 experts (SwiGLU ffn 512) + shared expert, top-10, 2-bit
+group-32 weights with fp16 scales, Zipf(1.1) popularity, frequency-ordered
+slots, verify windows of T = 1, 2, 3 and 4 tokens.  A step is one pass of the
+block (router, top-k, expert FFNs, shared expert, combine) over a batch of
+2048 rounds of the four windows (8192 windows, 20480 tokens), each window on
+the next of 32 independent layer copies (16 GB of weights, far above the
+126 MB L2) with fresh tokens.  The step is captured as one CUDA graph and
+replayed; the timed region holds exactly K steps, bracketed by a barrier and
+device syncs, timed with CUDA events, max over ranks.  The same line carries
+the metric's other half, the 8192-token prefill chunk (config of its own,
+timed the same way), as a `prefill` object.  One process per GPU; ranks run
+independent replicas (no collective on the data path).
 
 Prints one JSON line (rank 0).
 """
@@ -43,6 +46,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--layers", type=int, default=32, help="independent layer copies rotated")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-prefill", action="store_true",
+                   help="decode workload only (no prefill object in the line)")
+    p.add_argument("--prefill-steps", type=int, default=20)
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     return p.parse_args()
 
@@ -186,6 +192,14 @@ def measured_traffic(name: str):
 
 # ------------------------------------------------------------------ decode
 DECODE_WINDOWS = (1, 2, 3, 4)
+DECODE_ROUNDS = 2048        # rounds of the four windows in one step of the decode bench
+PREFILL_LAUNCHES = 11       # split router, router GEMM, top-k, prep, hist, scan, scatter,
+                            # gather, GEMM1, GEMM2, combine per 8192-token chunk
+WORKLOAD_DECODE = ("decode single layer: d=2048, 512 experts ffn=512 + shared ffn=512, top-10, "
+                   "2-bit g32 fp16 scales, Zipf(1.1) popularity, frequency-ordered slots; "
+                   "verify windows T=1,2,3,4")
+WORKLOAD_PREFILL = ("prefill chunk single layer: 8192 tokens, d=2048, 512 experts ffn=512 + "
+                    "shared ffn=512, top-10, 2-bit g32, router bias N(0,0.5)")
 
 
 def expert_bytes(shape) -> int:
@@ -211,6 +225,9 @@ def oracle_cpu_baseline(layer_cpu, windows, seconds, seed=777):
 
 
 def bench_decode(args, rank, world, local):
+    """The headline line: the decode layer (windows of 1..4 tokens) as `value`,
+    with the 8192-token prefill chunk of the same metric in a `prefill` object."""
+    import numpy as np
     import torch
 
     from routed_expert_ffn_06_b200 import moe, synth
@@ -220,59 +237,71 @@ def bench_decode(args, rank, world, local):
     wl = synth.WORKLOADS["decode"]
     sh = wl["shape"]
     NL = args.layers
-    K = args.steps if args.steps is not None else 20000
-    W = args.warmup if args.warmup is not None else 200
-    G = 500                      # steps per captured graph
+    K = args.steps if args.steps is not None else 20
+    W = args.warmup if args.warmup is not None else 5
+    R = DECODE_ROUNDS                      # rounds of the four windows per step
+    nwin = len(DECODE_WINDOWS)
+    ntok_step = R * sum(DECODE_WINDOWS)
     t_gen = time.time()
     layers = [synth.make_layer(sh, seed=rank * 1000 + i, layer=i, device=dev, bias=wl["bias"],
                                slot=wl["slot"]) for i in range(NL)]
     t_gen = time.time() - t_gen
     structs = [moe.make_layer_struct(l) for l in layers]
     ws = moe.alloc_workspace(structs[0], max(DECODE_WINDOWS))
-    nwin = len(DECODE_WINDOWS)
-    ntok_step = sum(DECODE_WINDOWS)
-    # fresh tokens per step (G distinct steps per graph)
-    xs = [[synth.make_tokens(T, sh.d, seed=rank * 1000 + 7, step=s * nwin + i, device=dev)
-           for i, T in enumerate(DECODE_WINDOWS)] for s in range(G)]
-    ys = [torch.empty(max(DECODE_WINDOWS), sh.d, dtype=torch.bfloat16, device=dev)
-          for _ in range(nwin)]
-    ids = [[torch.empty(T, sh.k, dtype=torch.int32, device=dev) for T in DECODE_WINDOWS]
-           for _ in range(G)]
-    wts = [[torch.empty(T, sh.k, dtype=torch.float32, device=dev) for T in DECODE_WINDOWS]
-           for _ in range(G)]
+    # fresh tokens for every window of a step
+    xs = [[synth.make_tokens(T, sh.d, seed=rank * 1000 + 7, step=r * nwin + i, device=dev)
+           for i, T in enumerate(DECODE_WINDOWS)] for r in range(R)]
+    ys = [torch.empty(T, sh.d, dtype=torch.bfloat16, device=dev) for T in DECODE_WINDOWS]
     stream = torch.cuda.Stream(device=dev)
 
-    def enqueue_step(s, events=None):
-        for i, T in enumerate(DECODE_WINDOWS):
-            L = structs[(s * nwin + i) % NL]
-            moe.moe_route_topk(L, xs[s][i], T, 0, None, ids[s][i], wts[s][i], ws, stream)
-            if events is not None:
-                events[s][i][0].record(stream)
-            moe.moe_expert_ffn_decode(L, xs[s][i], T, ids[s][i], wts[s][i], ys[i], 0, ws, stream)
-            if events is not None:
-                events[s][i][1].record(stream)
+    def layer_of(r, i):
+        return structs[(r * nwin + i) % NL]
 
-    # eager pass: sets kernel attributes, fills routing for the byte counts
+    def enqueue_step():
+        for r in range(R):
+            for i, T in enumerate(DECODE_WINDOWS):
+                moe.moe_block_forward(layer_of(r, i), xs[r][i], T, ys[i], 0, ws, stream)
+
+    # eager pass: kernel attributes and tensor maps set up; routing of every
+    # window for the byte counts (the block forward records it in the workspace)
+    ids_all = [[None] * nwin for _ in range(R)]
+    wts_all = [[None] * nwin for _ in range(R)]
+    eb = expert_bytes(sh)
     with torch.cuda.stream(stream):
-        for s in range(G):
-            enqueue_step(s)
+        for r in range(R):
+            for i, T in enumerate(DECODE_WINDOWS):
+                ids = torch.empty(T, sh.k, dtype=torch.int32, device=dev)
+                wts = torch.empty(T, sh.k, dtype=torch.float32, device=dev)
+                moe.moe_route_topk(layer_of(r, i), xs[r][i], T, 0, None, ids, wts, ws, stream)
+                ids_all[r][i], wts_all[r][i] = ids, wts
+        enqueue_step()
     stream.synchronize()
     st, code = moe.moe_workspace_error(ws, stream)
     if st != 0:
         raise RuntimeError(f"device error word {code:#x}")
-    eb = expert_bytes(sh)
+    uniq = [[int(torch.unique(ids_all[r][i]).numel()) for i in range(nwin)] for r in range(R)]
+    U_mean = {str(T): round(float(np.mean([uniq[r][i] for r in range(R)])), 2)
+              for i, T in enumerate(DECODE_WINDOWS)}
+    # fitted Zipf exponent of the realised selection counts (all windows, all
+    # layer copies, experts ranked by their own layer's popularity profile)
+    counts = np.zeros(sh.E)
+    for r in range(R):
+        for i in range(nwin):
+            rank_of = layers[(r * nwin + i) % NL].rank.numpy() - 1
+            np.add.at(counts, rank_of[ids_all[r][i].cpu().numpy().ravel()], 1)
+    top = np.sort(counts)[::-1][:200]
+    top = top[top > 0]
+    zipf_s = float(-np.polyfit(np.log(np.arange(1, len(top) + 1)), np.log(top), 1)[0])
+    # algorithmic bytes of one step: per window the router (E x d fp32), the
+    # window's unique experts and the shared expert, the tokens in and out
+    step_bytes = sum(sh.E * sh.d * 4 + (uniq[r][i] + 1) * eb + 2 * T * sh.d * 2
+                     for r in range(R) for i, T in enumerate(DECODE_WINDOWS))
 
-    # graphs: one of G steps
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
-        for s in range(G):
-            enqueue_step(s)
-    reps_w = max(1, W // G)
-    reps = max(1, K // G)
-    K = reps * G
-    W = reps_w * G
+        enqueue_step()
     with torch.cuda.stream(stream):
-        for _ in range(reps_w):
+        for _ in range(W):
             g.replay()
     stream.synchronize()
     barrier(world)
@@ -282,126 +311,140 @@ def bench_decode(args, rank, world, local):
     with ClockSampler(local) as clk:
         with torch.cuda.stream(stream):
             e0.record(stream)
-            for _ in range(reps):
+            for _ in range(K):
                 g.replay()
             e1.record(stream)
         stream.synchronize()
     torch.cuda.synchronize()
     barrier(world)
-    ms = e0.elapsed_time(e1)
-    ms = max_over_ranks(ms, world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
     clocks = clk.summary()
     value = K * ntok_step * world / (ms / 1e3)
+    peaks = measured_peaks()
+    layer_gbs = step_bytes / (ms / K / 1e3) / 1e9
+    del g
 
-    # component timing: the expert step alone (moe_expert_ffn_decode on the
-    # routing of the eager pass), one graph per window size replayed between two
-    # events on the launching stream; events inside a graph would break the
-    # programmatic overlap of its kernels, so none are recorded there
-    Gc = min(G, 200)
-    win_bytes = [[0] * nwin for _ in range(G)]
-    for s in range(G):
-        for i, T in enumerate(DECODE_WINDOWS):
-            U = int(torch.unique(ids[s][i]).numel())
-            win_bytes[s][i] = (U + 1) * eb + 2 * T * sh.d * 2
-    per_T = {}
-    exp_ms_total, exp_bytes = 0.0, 0
-    R = 4
+    # the expert step alone (moe_expert_ffn_decode on the eager pass's routing:
+    # expert kernel + combine), one graph per window size, events around the
+    # replays on the launching stream (events inside a graph would break the
+    # programmatic overlap of its kernels)
+    per_T, exp_ms_total, exp_bytes, n_exp = {}, 0.0, 0, 0
+    Rc = min(R, 256)
     for i, T in enumerate(DECODE_WINDOWS):
         gt = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gt, stream=stream):
-            for s in range(Gc):
-                L = structs[(s * nwin + i) % NL]
-                moe.moe_expert_ffn_decode(L, xs[s][i], T, ids[s][i], wts[s][i], ys[i], 0, ws, stream)
+            for r in range(Rc):
+                moe.moe_expert_ffn_decode(layer_of(r, i), xs[r][i], T, ids_all[r][i],
+                                          wts_all[r][i], ys[i], 0, ws, stream)
         c0 = torch.cuda.Event(enable_timing=True)
         c1 = torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             gt.replay()
             c0.record(stream)
-            for _ in range(R):
+            for _ in range(4):
                 gt.replay()
             c1.record(stream)
         stream.synchronize()
-        t_ms = c0.elapsed_time(c1) / R
-        per_T[str(T)] = round(1e3 * t_ms / Gc, 2)
+        t_ms = c0.elapsed_time(c1) / 4
+        per_T[str(T)] = round(1e3 * t_ms / Rc, 2)
         exp_ms_total += t_ms
-        exp_bytes += sum(win_bytes[s][i] for s in range(Gc))
+        exp_bytes += sum((uniq[r][i] + 1) * eb + 2 * T * sh.d * 2 for r in range(Rc))
+        n_exp += Rc
         del gt
     achieved = exp_bytes / (exp_ms_total / 1e3) / 1e9
-    peaks = measured_peaks()
 
-    # end to end through the public call with host buffers
-    Ke = min(K, 2000)
-    xh = [[x.cpu().pin_memory() for x in xs[s]] for s in range(G)]
-    yh = [torch.empty(T, sh.d, dtype=torch.bfloat16).pin_memory() for T in DECODE_WINDOWS]
+    # end to end through the public call: every window's tokens copied from
+    # pinned host memory, the block forward, the output copied back; captured
+    # as one CUDA graph per step (the copies are nodes of the graph)
+    xh = [[x.cpu().pin_memory() for x in xs[r]] for r in range(R)]
+    yh = [[torch.empty(T, sh.d, dtype=torch.bfloat16).pin_memory() for T in DECODE_WINDOWS]
+          for _ in range(R)]
     xd = [torch.empty(T, sh.d, dtype=torch.bfloat16, device=dev) for T in DECODE_WINDOWS]
-    ysd = [torch.empty(T, sh.d, dtype=torch.bfloat16, device=dev) for T in DECODE_WINDOWS]
+    Ke = min(K, 4)
+    ge = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ge, stream=stream):
+        for r in range(R):
+            for i, T in enumerate(DECODE_WINDOWS):
+                xd[i].copy_(xh[r][i], non_blocking=True)
+                moe.moe_block_forward(layer_of(r, i), xd[i], T, ys[i], 0, ws, stream)
+                yh[r][i].copy_(ys[i], non_blocking=True)
+    with torch.cuda.stream(stream):
+        ge.replay()
+    stream.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     f0 = torch.cuda.Event(enable_timing=True)
     f1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         f0.record(stream)
-        for s in range(Ke):
-            for i, T in enumerate(DECODE_WINDOWS):
-                L = structs[(s * nwin + i) % NL]
-                xd[i].copy_(xh[s % G][i], non_blocking=True)
-                moe.moe_block_forward(L, xd[i], T, ysd[i], 0, ws, stream)
-                yh[i].copy_(ysd[i], non_blocking=True)
+        for _ in range(Ke):
+            ge.replay()
         f1.record(stream)
     stream.synchronize()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
     e2e_value = Ke * ntok_step * world / (e2e_ms / 1e3)
+    del ge
 
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": K, "warmup": W, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
+        "steps": K, "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic (seeded; random-init weights of the stated architecture)",
-        "config": {"workload": "decode single layer: d=2048, 512 experts ffn=512 + shared "
-                               "ffn=512, top-10, 2-bit g32 fp16 scales, Zipf(1.1) popularity, "
-                               "frequency-ordered slots; windows T=1,2,3,4 per step",
+        "config": {"workload": WORKLOAD_DECODE,
+                   "step": f"{R} rounds of the T=1,2,3,4 windows ({R * nwin} windows), each window "
+                           f"on the next of {NL} layer copies with fresh tokens",
                    "tokens_per_step": ntok_step, "layer_copies": NL,
                    "l2": "inputs larger than L2 (32 layer copies rotated, "
                          f"{NL * (sh.E * eb + sh.E * sh.d * 4) / 1e9:.1f} GB)",
-                   "parallelism": f"replicas x{world}", "graph_steps": G,
+                   "parallelism": f"replicas x{world}",
                    "mma": "f16 x f16 -> f32 (weights dequantised in registers)",
+                   "unique_experts_per_window": U_mean, "zipf_s_fitted": round(zipf_s, 3),
                    "weights_gen_s": round(t_gen, 1)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "traffic": measured_traffic("decode_expert_step"), "peak_src": peaks["src"],
-                     "kernel": "expert step (decode_gu + decode_dn per moe_expert_ffn_decode call)",
-                     "bytes_per_launch": round(exp_bytes / (Gc * nwin)),
+                     "kernel": "expert step (decode_expert_kernel + decode_combine_kernel per "
+                               "moe_expert_ffn_decode call)",
+                     "bytes_per_launch": round(exp_bytes / n_exp),
                      "us_per_launch_by_T": per_T,
                      "timing": "graphs of expert steps only, events around the replays"},
+        "layer_roofline": {"bound": "hbm", "achieved": round(layer_gbs, 1),
+                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": round(layer_gbs / peaks["hbm_gbs"], 4),
+                           "bytes_per_step": step_bytes,
+                           "us_per_window": round(1e3 * ms / K / (R * nwin), 3),
+                           "what": "whole block (router, experts, combine) over the timed steps"},
         "clocks": clocks,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": ntok_step * sh.d * 2, "d2h_bytes_per_step": ntok_step * sh.d * 2,
-                "steps": Ke, "path": "moe_block_forward via the ctypes binding, pinned host x/y"},
-        "gpu_launches": K * nwin * 3,   # router, gate/up, down per window
+                "steps": Ke,
+                "path": "moe_block_forward via the ctypes binding with each window's pinned-host "
+                        "copies in and out, captured as one CUDA graph per step"},
+        "gpu_launches": K * R * nwin * 3,   # router, expert, combine per window
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = oracle_cpu_baseline(layers[0].to("cpu"), DECODE_WINDOWS,
                                                args.cpu_seconds)
         res["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cores,
                                "kind": "oracle", "sample": sample}
+    del layers, structs, xs
+    torch.cuda.empty_cache()
+    if not args.no_prefill:
+        res["prefill"] = measure_prefill(args, rank, world, local, K=args.prefill_steps, W=3)
+        res["gpu_launches"] += res["prefill"]["gpu_launches"]
     return res
 
 
-# ----------------------------------------------------------------- prefill
-def bench_prefill(args, rank, world, local):
+def measure_prefill(args, rank, world, local, K, W):
     """One layer, 8192-token chunk, 2-bit, router bias ~ N(0, 0.5).  A step is
-    one block forward over the chunk (router, top-k, bucketing, grouped
-    GEMMs, shared expert, combine); two layer copies alternate."""
+    one block forward over the chunk (router, top-k, bucketing, grouped GEMMs,
+    shared expert, combine); two layer copies alternate."""
     import torch
 
     from routed_expert_ffn_06_b200 import moe, synth
     dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    moe.load()
     wl = synth.WORKLOADS["prefill"]
     sh, T = wl["shape"], wl["T"]
-    K = args.steps if args.steps is not None else 40
-    W = args.warmup if args.warmup is not None else 5
     NL = 2
     layers = [synth.make_layer(sh, seed=rank * 1000 + i, layer=i, device=dev, bias=wl["bias"],
                                bias_std=wl["bias_std"], slot=wl["slot"]) for i in range(NL)]
@@ -444,11 +487,11 @@ def bench_prefill(args, rank, world, local):
         stream.synchronize()
     barrier(world)
     ms = max_over_ranks(e0.elapsed_time(e1), world)
-    exp_ms = sum(ev[0].elapsed_time(ev[1]) for ev in evs) / K
+    exp_ms = max_over_ranks(sum(ev[0].elapsed_time(ev[1]) for ev in evs) / K, world)
     peaks = measured_peaks()
     flops = 2.0 * T * (sh.k + 1) * 3 * sh.F * sh.d          # gate/up + down, routed + shared
     achieved = flops / (exp_ms / 1e3) / 1e12
-    # e2e: host chunk in, host output out, public block call
+    # e2e: the chunk from pinned host memory, the public block call, back to the host
     xh = xs[0].cpu().pin_memory()
     yh = torch.empty(T, sh.d, dtype=torch.bfloat16).pin_memory()
     xd = torch.empty_like(xs[0])
@@ -467,16 +510,9 @@ def bench_prefill(args, rank, world, local):
     stream.synchronize()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
     res = {
-        "metric": METRIC, "value": round(K * T * world / (ms / 1e3), 1), "unit": "tokens/s",
-        "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms / K, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-        "data": "synthetic (seeded; random-init weights of the stated architecture)",
-        "config": {"workload": "prefill chunk single layer: 8192 tokens, d=2048, 512 experts "
-                               "ffn=512 + shared ffn=512, top-10, 2-bit g32, router bias N(0,0.5)",
-                   "tokens_per_step": T, "layer_copies": NL,
-                   "l2": "inputs larger than L2 (504 MB packed weights per layer)",
-                   "parallelism": f"replicas x{world}",
-                   "mma": "tcgen05 kind::f16, fp16 operands (weights dequantised to smem), fp32 TMEM"},
+        "workload": WORKLOAD_PREFILL, "value": round(K * T * world / (ms / 1e3), 1),
+        "unit": "tokens/s", "steps": K, "warmup": W, "ms_per_step": round(ms / K, 4),
+        "tokens_per_step": T,
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / peaks["bf16_tflops"], 4),
@@ -489,8 +525,7 @@ def bench_prefill(args, rank, world, local):
         "e2e": {"value": round(Ke * T * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * sh.d * 2, "d2h_bytes_per_step": T * sh.d * 2,
                 "steps": Ke, "path": "moe_block_forward via the ctypes binding, pinned host x/y"},
-        # split router, router GEMM, top-k, prep, hist, scan, scatter, gather, GEMM1, GEMM2, combine
-        "gpu_launches": K * 11,
+        "gpu_launches": K * PREFILL_LAUNCHES,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -504,6 +539,32 @@ def bench_prefill(args, rank, world, local):
         res["cpu_baseline"] = {"value": round(n_tok / dt, 3), "unit": "tokens/s",
                                "cores": oracle.num_threads(), "kind": "oracle",
                                "sample": f"{n_tok} of the chunk's 8192 tokens"}
+    return res
+
+
+def bench_prefill(args, rank, world, local):
+    """--workload prefill: the prefill chunk as the line's value."""
+    import torch
+    torch.cuda.set_device(local)
+    from routed_expert_ffn_06_b200 import moe
+    moe.load()
+    K = args.steps if args.steps is not None else 40
+    W = args.warmup if args.warmup is not None else 5
+    p = measure_prefill(args, rank, world, local, K, W)
+    res = {"metric": METRIC, "value": p["value"], "unit": "tokens/s", "n_gpus": world,
+           "steps": K, "warmup": W, "ms_per_step": p["ms_per_step"], "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+           "data": "synthetic (seeded; random-init weights of the stated architecture)",
+           "config": {"workload": WORKLOAD_PREFILL, "tokens_per_step": p["tokens_per_step"],
+                      "layer_copies": 2,
+                      "l2": "inputs larger than L2 (504 MB packed weights per layer)",
+                      "parallelism": f"replicas x{world}",
+                      "mma": "tcgen05 kind::f16, fp16 operands (weights dequantised to smem), "
+                             "fp32 TMEM"},
+           "roofline": p["roofline"], "clocks": p["clocks"], "e2e": p["e2e"],
+           "gpu_launches": p["gpu_launches"]}
+    if "cpu_baseline" in p:
+        res["cpu_baseline"] = p["cpu_baseline"]
     return res
 
 
@@ -764,20 +825,19 @@ def run_reference(args, rank, world):
         return None
     import oracle
     from routed_expert_ffn_06_b200 import synth
-    K = min(args.steps if args.steps is not None else 5, 20)
-    W = min(args.warmup if args.warmup is not None else 1, 3)
+    K = args.steps if args.steps is not None else 20
+    W = args.warmup if args.warmup is not None else 5
     if args.workload == "prefill":
         wl = synth.WORKLOADS["prefill"]
         layer = synth.make_layer(wl["shape"], seed=0, device="cpu", bias=wl["bias"],
                                  bias_std=wl["bias_std"], slot=wl["slot"])
         OL = oracle.OracleLayer(layer)
         x = synth.make_tokens(wl["T"], wl["shape"].d, seed=3, step=0)
-        per = 16   # tokens of the 8192 chunk per step
+        per = 8    # tokens of the 8192 chunk per step
 
         def step(s):
             OL.block_forward(x, rows=list(range((s * per) % wl["T"], (s * per) % wl["T"] + per)))
-        workload = ("prefill chunk single layer: 8192 tokens, d=2048, 512 experts ffn=512 + "
-                    "shared ffn=512, top-10, 2-bit g32, router bias N(0,0.5)")
+        workload = WORKLOAD_PREFILL
         sample = f"{per} of the chunk's tokens per step"
         tok = per
     elif args.workload in ("stack", "mix"):
@@ -806,9 +866,8 @@ def run_reference(args, rank, world):
         def step(s):
             for i, T in enumerate(DECODE_WINDOWS):
                 OL.block_forward(synth.make_tokens(T, wl["shape"].d, seed=7, step=s * 4 + i))
-        workload = ("decode single layer: d=2048, 512 experts ffn=512 + shared ffn=512, top-10, "
-                    "2-bit g32, Zipf(1.1); windows T=1,2,3,4 per step")
-        sample = f"{K} steps of 4 windows (10 tokens)"
+        workload = WORKLOAD_DECODE
+        sample = "one round of the T=1,2,3,4 windows (10 tokens) per step"
         tok = sum(DECODE_WINDOWS)
     for s in range(W):
         step(s)

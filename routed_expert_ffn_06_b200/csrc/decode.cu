@@ -57,6 +57,7 @@ struct ExpList {
 // are replaced by 0 and flagged, so no later address leaves the expert array.
 __device__ void expert_list_prologue(const LayerDev& L, ExpList* s, int* slot_s, int* first,
                                      Control* ctl) {
+#pragma unroll 1
   for (int e = threadIdx.x; e < L.E; e += blockDim.x) {
     int sl = L.slot[e];
     if (sl < 0 || sl >= L.E) {
@@ -66,6 +67,7 @@ __device__ void expert_list_prologue(const LayerDev& L, ExpList* s, int* slot_s,
     slot_s[e] = sl;
     first[e] = 0x7FFFFFFF;
   }
+#pragma unroll 1
   for (int i = threadIdx.x; i < kMaxExp * kMaxDecodeT; i += blockDim.x) (&s->w[0][0])[i] = 0.f;
 }
 
@@ -288,10 +290,10 @@ __host__ __device__ inline DecSmem dec_smem(int d, int E, int bits, int nslots) 
   m.xs = o;                                        // B fragments of the tokens, per group
   o += (size_t)nG * 32 * 16;
   m.corr = o;                                      // 2-bit offset-form correction [group][token]
-  o += (size_t)nG * kMaxDecodeT * sizeof(float);
+  o += (size_t)nG * kMaxDecodeT * sizeof(float);   // (xs and corr: one bulk copy, in this order)
   o = (o + 15) & ~size_t(15);
-  m.part = o;                                      // gate/up partial sums [warp][lane][4]
-  o += (size_t)kDecWarps * 32 * 4 * sizeof(float);
+  m.part = o;                                      // gate/up partial sums [warp][tile][lane][4]
+  o += (size_t)kDecWarps * 2 * 32 * 4 * sizeof(float);
   m.hfrag = o;                                     // hidden slice as down B fragments [lane][4]
   o += 32 * 4 * sizeof(uint32_t);
   o = (o + 127) & ~size_t(127);
@@ -331,7 +333,7 @@ __device__ __forceinline__ ExpSrc expert_src(const LayerDev& L, bool shared, int
 // slice s of expert `src` into `dst`; completion on `bar` (one arrival plus the
 // piece's bytes).  One thread.
 template <int BITS>
-__device__ __forceinline__ void issue_piece(const DecMaps& maps, const LayerDev& L, const ExpSrc& src,
+__device__ __noinline__ void issue_piece(const DecMaps& maps, const LayerDev& L, const ExpSrc& src,
                                             int s, int kind, unsigned char* dst, uint64_t* bar) {
   const int d = L.d, nG = d / kGroup, gb = group_bytes(BITS);
   mbar_arrive_expect_tx(bar, dec_piece_bytes(d, BITS));
@@ -357,15 +359,24 @@ __device__ __forceinline__ void issue_piece(const DecMaps& maps, const LayerDev&
 // first, then each routed expert's in first-occurrence order of the window);
 // unit n runs on CTA n % G.  NRT: output-row tiles per warp (d / 256, rounded
 // up to 8 or 16).
+//
+// Warp roles inside a unit: gate/up -- warp w takes matrix w / 8 (Wg, Wu) and
+// the K-eighth w % 8 of both 16-row tiles of the slice, so each token fragment
+// it loads serves two tiles; the eight partial sums of a (matrix, tile) are
+// added in warp order.  Down -- warp w takes the output-row tiles w, w+16, ...
+// of the Wd group column and keeps their sums in registers across units.
+// The tokens' B fragments (and, for 2-bit, the offset-form corrections) come
+// precomputed from the router kernel: one bulk copy.
 // At most 88 registers per thread, so that a router or combine CTA can stay
 // resident beside it (programmatic dependent launch overlaps the kernels).
 template <int BITS, int NRT>
 __global__ void __maxnreg__(88)
-    decode_expert_kernel(const __grid_constant__ DecMaps maps, LayerDev L,
-                         const uint16_t* __restrict__ x, int T, const float* __restrict__ logits,
-                         const int32_t* __restrict__ ids_in, const float* __restrict__ w_in,
-                         int32_t* __restrict__ ids_out, float* __restrict__ w_out,
-                         float* __restrict__ partial, uint32_t flags, Control* ctl, int nslots) {
+    decode_expert_kernel(const __grid_constant__ DecMaps maps, const __grid_constant__ LayerDev L,
+                         const unsigned char* __restrict__ xfrag, int T,
+                         const float* __restrict__ logits, const int32_t* __restrict__ ids_in,
+                         const float* __restrict__ w_in, int32_t* __restrict__ ids_out,
+                         float* __restrict__ w_out, float* __restrict__ partial, uint32_t flags,
+                         Control* ctl, int nslots) {
   extern __shared__ __align__(128) unsigned char smem[];
   const DecSmem m = dec_smem(L.d, L.E, BITS, nslots);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + m.bars);
@@ -374,12 +385,12 @@ __global__ void __maxnreg__(88)
   int* slot_s = first + L.E;
   int32_t* sel_ids = reinterpret_cast<int32_t*>(smem + m.sel);
   float* sel_w = reinterpret_cast<float*>(sel_ids + kMaxDecodeT * 16);
-  uint4* xs = reinterpret_cast<uint4*>(smem + m.xs);
-  float* corr = reinterpret_cast<float*>(smem + m.corr);
+  const uint4* xs = reinterpret_cast<const uint4*>(smem + m.xs);
+  const float* corr = reinterpret_cast<const float*>(smem + m.corr);
   float* part = reinterpret_cast<float*>(smem + m.part);
   __half* hfrag = reinterpret_cast<__half*>(smem + m.hfrag);
   unsigned char* slots = smem + m.slots;
-  __shared__ float inv_rms[kMaxDecodeT];
+  __shared__ __align__(8) uint64_t xbar;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int d = L.d, nG = d / kGroup, gb = group_bytes(BITS);
@@ -390,6 +401,7 @@ __global__ void __maxnreg__(88)
 
   if (tid == 0) {
     for (int s = 0; s < nslots; ++s) mbar_init(&full[s], 1);
+    mbar_init(&xbar, 1);
     fence_barrier_init();
   }
   // the tensor-map descriptors in use into the TMA unit's cache
@@ -400,100 +412,44 @@ __global__ void __maxnreg__(88)
   expert_list_prologue(L, list, slot_s, first, ctl);
   __syncthreads();
 
-  // The shared expert's units do not depend on the routing: request them
-  // before waiting for the router.
+  // The shared expert's first unit does not depend on the routing: request it
+  // before waiting for the router.  Until the first unit's slices have landed
+  // only one unit is in flight, so that it is not queued behind the whole
+  // GPU's requests; then the ring fills up.
   int issued = 0;   // pieces requested (thread 0)
-  if (tid == 0 && sh_units > 0) {
-    for (int p = 0; p < nslots; ++p) {
-      const int n = blockIdx.x + (p / 3) * G;
-      if (n >= sh_units) break;
-      issue_piece<BITS>(maps, L, expert_src(L, true, 0), n, p % 3, slot_ptr(p), &full[p % nslots]);
+  int cap = 3;      // pieces allowed ahead of the consumer
+  if (tid == 0 && sh_units > (int)blockIdx.x) {
+    for (int p = 0; p < 3 && p < nslots; ++p) {
+      issue_piece<BITS>(maps, L, expert_src(L, true, 0), blockIdx.x, p, slot_ptr(p), &full[p]);
       issued = p + 1;
     }
   }
 
-  pdl_wait();   // router logits (or the given routing) and x are complete
+  pdl_wait();   // router logits (or the given routing) and the token fragments are complete
   pdl_launch_dependents();
+  if (tid == 0) {
+    const uint32_t xb = (uint32_t)nG * (32 * 16 + kMaxDecodeT * 4);
+    mbar_arrive_expect_tx(&xbar, xb);
+    bulk_g2s(smem + m.xs, xfrag, xb, &xbar);
+  }
 
-  // ---- routing of the window (warps 0..T-1) and the tokens' B fragments
-  //      (the other warps, then everyone)
+  // ---- routing of the window (warps 0..T-1 select from the logits)
   if (logits) {
-    if (warp < T)
-      warp_topk(logits + (size_t)warp * L.E, L.E, L.k, sel_ids + warp * L.k, sel_w + warp * L.k,
-                ctl, flags & MOE_F_DEBUG);
+    if (warp < T) {
+      const float* row = logits + (size_t)warp * L.E;
+      if (L.E <= 512)
+        warp_topk_n<16>(row, L.E, L.k, sel_ids + warp * L.k, sel_w + warp * L.k, ctl, flags & MOE_F_DEBUG);
+      else
+        warp_topk_n<32>(row, L.E, L.k, sel_ids + warp * L.k, sel_w + warp * L.k, ctl, flags & MOE_F_DEBUG);
+    }
   } else {
+#pragma unroll 1
     for (int i = tid; i < T * L.k; i += blockDim.x) {
       sel_ids[i] = __ldcg(ids_in + i);
       sel_w[i] = __ldcg(w_in + i);
     }
   }
-  const bool pn = flags & MOE_F_PRENORM;
-  if (pn && warp >= kDecWarps - kMaxDecodeT && warp - (kDecWarps - kMaxDecodeT) < T) {
-    const int t = warp - (kDecWarps - kMaxDecodeT);
-    float ss = 0.f;
-    for (int i = lane * 8; i < d; i += 256) {
-      const uint4 v = *reinterpret_cast<const uint4*>(x + (size_t)t * d + i);
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float a = __uint_as_float(w4[j] << 16), b = __uint_as_float(w4[j] & 0xFFFF0000u);
-        ss += a * a + b * b;
-      }
-    }
-    ss = warp_sum(ss);
-    if (lane == 0) inv_rms[t] = rsqrtf(ss / (float)d + kRmsEps);
-  }
   __syncthreads();
-  // one (token n, group c) pair per thread: 32 values -> the 16-byte B
-  // fragments of lanes 4n .. 4n+3 (pair m of lane 4n+t = columns 8m+2t, +1).
-  // fp16 operands: values outside the fp16 range are flagged (always on).
-  {
-    bool bad = false;
-    for (int pidx = tid; pidx < kMaxDecodeT * nG; pidx += blockDim.x) {
-      const int c = pidx >> 3, n = pidx & 7;
-      uint4 out[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
-                      make_uint4(0, 0, 0, 0)};
-      float cs = 0.f;
-      if (n < T) {
-        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)n * d + 32 * c);
-        uint32_t w[16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 v = src[q];
-          w[4 * q] = v.x;
-          w[4 * q + 1] = v.y;
-          w[4 * q + 2] = v.z;
-          w[4 * q + 3] = v.w;
-        }
-        const float sc = pn ? inv_rms[n] : 1.f;
-        uint32_t h2[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {   // w[q] holds columns 2q, 2q+1 = 8m + 2t (+1), q = 4m + t
-          float v0 = __uint_as_float(w[q] << 16), v1 = __uint_as_float(w[q] & 0xFFFF0000u);
-          if (pn) {
-            v0 = __bfloat162float(__float2bfloat16_rn(v0 * sc));
-            v1 = __bfloat162float(__float2bfloat16_rn(v1 * sc));
-          }
-          bad |= !(fabsf(v0) <= 65504.f) || !(fabsf(v1) <= 65504.f);
-          if (BITS == 2) {
-            // offset form: B = x / 4^m; correction sum B * (1024 + 2 * 4^m)
-            const float inv = 1.f / (float)(1 << (2 * (q >> 2)));
-            const __half2 bh = __floats2half2_rn(v0 * inv, v1 * inv);
-            h2[q] = h2_as_u32(bh);
-            cs += (__low2float(bh) + __high2float(bh)) * (1024.f + 2.f * (float)(1 << (2 * (q >> 2))));
-          } else {
-            h2[q] = h2_as_u32(__floats2half2_rn(v0, v1));
-          }
-        }
-#pragma unroll
-        for (int t = 0; t < 4; ++t) out[t] = make_uint4(h2[t], h2[4 + t], h2[8 + t], h2[12 + t]);
-      }
-      corr[c * kMaxDecodeT + n] = cs;
-#pragma unroll
-      for (int t = 0; t < 4; ++t) xs[c * 32 + n * 4 + t] = out[t];
-    }
-    if (bad) record_error(ctl, kErrNonFinite, 0x600);
-  }
   if (warp == 0) build_expert_list(sel_ids, sel_w, T, L, list, slot_s, first, ctl);
   __syncthreads();
   if (blockIdx.x == 0 && ids_out) {
@@ -522,7 +478,8 @@ __global__ void __maxnreg__(88)
     return n < sh_units ? 0 : (L.Fs > 0 ? 1 : 0) + (n - sh_units) / Fu;
   };
   auto refill = [&](int consumed) {   // thread 0: keep the ring full, in consumption order
-    while (issued < npieces && issued < consumed + nslots) {
+    const int lim = consumed + (cap < nslots ? cap : nslots);
+    while (issued < npieces && issued < lim) {
       int s;
       const ExpSrc src = unit_src(issued / 3, &s);
       issue_piece<BITS>(maps, L, src, s, issued % 3, slot_ptr(issued), &full[issued % nslots]);
@@ -530,37 +487,45 @@ __global__ void __maxnreg__(88)
     }
   };
   if (tid == 0) refill(0);
+  bool ok = mbar_wait(&xbar, 0, ctl, 0x600);
 
   float accd[NRT][4];
 #pragma unroll
   for (int i = 0; i < NRT; ++i) accd[i][0] = accd[i][1] = accd[i][2] = accd[i][3] = 0.f;
   const int ntiles = d / kTileRows;
-  const int mat = warp >> 3, tl = (warp >> 2) & 1, kq = warp & 3;
-  const int c0 = kq * nG / 4, c1 = (kq + 1) * nG / 4;
+  const int mat = warp >> 3, kq = warp & 7;
+  const int c0 = kq * nG / 8, c1 = (kq + 1) * nG / 8;
   int j = 0;
   for (; j < my; ++j) {
     const int pg = 3 * j, pu = pg + 1, pd = pg + 2;
-    bool ok = mbar_wait(&full[pg % nslots], (pg / nslots) & 1, ctl, 0x601);
+    ok = ok && mbar_wait(&full[pg % nslots], (pg / nslots) & 1, ctl, 0x601);
     ok = ok && mbar_wait(&full[pu % nslots], (pu / nslots) & 1, ctl, 0x602);
     if (!__syncthreads_and(ok)) break;
-    // gate/up: warp (mat, tile, K quarter)
+    if (j == 0 && tid == 0) {   // the first unit is here: let the ring fill
+      cap = nslots;
+      refill(0);
+    }
+    // gate/up: warp (matrix, K eighth), both tiles of the slice
     {
       const unsigned char* pc = slot_ptr(mat ? pu : pg);
-      const unsigned char* tb = pc + tl * tcb;
-      const __half* sc = reinterpret_cast<const __half*>(pc + 2 * tcb) + tl * kTileRows * nG;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+      const __half* sc = reinterpret_cast<const __half*>(pc + 2 * tcb);
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
       for (int c = c0; c < c1; ++c) {
         const uint4 xf = xs[c * 32 + lane];
         const uint32_t b[4] = {xf.x, xf.y, xf.z, xf.w};
         if (BITS == 2) {
           const float2 cr = *reinterpret_cast<const float2*>(corr + c * kMaxDecodeT + 2 * (lane & 3));
-          group_mma_2b_offset(tb, sc, c, b, cr, acc);
+          group_mma_2b_offset(pc, sc, c, b, cr, a0);
+          group_mma_2b_offset(pc + tcb, sc + kTileRows * nG, c, b, cr, a1);
         } else {
-          group_mma<BITS>(tb, tb + nG * kTileRows * 8, sc, c, b, acc);
+          group_mma<BITS>(pc, pc + nG * kTileRows * 8, sc, c, b, a0);
+          group_mma<BITS>(pc + tcb, pc + tcb + nG * kTileRows * 8, sc + kTileRows * nG, c, b, a1);
         }
       }
-      *reinterpret_cast<float4*>(part + (warp * 32 + lane) * 4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      float4* pw = reinterpret_cast<float4*>(part) + (warp * 2) * 32 + lane;
+      pw[0] = make_float4(a0[0], a0[1], a0[2], a0[3]);
+      pw[32] = make_float4(a1[0], a1[1], a1[2], a1[3]);
     }
     __syncthreads();
     if (tid == 0) {   // the Wg and Wu slots are free
@@ -572,16 +537,18 @@ __global__ void __maxnreg__(88)
       const int htl = tid >> 7, ln = (tid >> 2) & 31, e = tid & 3;
       float gs = 0.f, us = 0.f;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        gs += part[((htl * 4 + q) * 32 + ln) * 4 + e];
-        us += part[((8 + htl * 4 + q) * 32 + ln) * 4 + e];
+      for (int q = 0; q < 8; ++q) {
+        gs += part[((q * 2 + htl) * 32 + ln) * 4 + e];
+        us += part[(((8 + q) * 2 + htl) * 32 + ln) * 4 + e];
       }
       const int row = (ln >> 2) + 8 * (e >> 1) + 16 * htl;   // hidden unit within the slice
       const int n = 2 * (ln & 3) + (e & 1);                   // token
       float h = 0.f;
       if (n < T) h = gs / (1.f + expf(-gs)) * us * list->w[unit_u(j)][n];
       if (!(fabsf(h) <= 65504.f)) record_error(ctl, kErrNonFinite, 0x603);
-      // down-projection B fragment: k = row, column = token
+      // down-projection B fragment: k = row, column = token; 2-bit offset
+      // form: the value divided by 4^(k / 8)
+      if (BITS == 2) h *= 1.f / (float)(1 << (2 * (row >> 3)));
       const int tp = (row & 7) >> 1, jj = row >> 3, hh = row & 1;
       hfrag[((n * 4 + tp) * 4 + jj) * 2 + hh] = __float2half_rn(h);
     }
@@ -593,10 +560,33 @@ __global__ void __maxnreg__(88)
       const uint32_t b[4] = {hb.x, hb.y, hb.z, hb.w};
       const unsigned char* pp = slot_ptr(pd);
       const __half* dsc = reinterpret_cast<const __half*>(pp + gb * d);
+      if (BITS == 2) {
+        // offset-form correction of token g: sum over the group of
+        // B * (1024 + 2 * 4^m); this lane holds 8 of the 32 values (k = 2t +
+        // {0,1} + 8m), the four lanes t of the row group hold all of them
+        float cs = 0.f;
 #pragma unroll
-      for (int i = 0; i < NRT; ++i) {
-        const int r = warp + kDecWarps * i;
-        if (r < ntiles) group_mma<BITS>(pp + r * 128, pp + 8 * d + r * 64, dsc + r * kTileRows, 0, b, accd[i]);
+        for (int q = 0; q < 4; ++q) {
+          const __half2 v = u32_as_h2(b[q]);
+          cs += (__low2float(v) + __high2float(v)) * (1024.f + 2.f * (float)(1 << (2 * q)));
+        }
+        cs += __shfl_xor_sync(0xffffffffu, cs, 1);
+        cs += __shfl_xor_sync(0xffffffffu, cs, 2);
+        const int t = lane & 3;
+        const float2 cr = make_float2(__shfl_sync(0xffffffffu, cs, 8 * t),
+                                      __shfl_sync(0xffffffffu, cs, 8 * t + 4));
+#pragma unroll
+        for (int i = 0; i < NRT; ++i) {
+          const int r = warp + kDecWarps * i;
+          if (r < ntiles) group_mma_2b_offset(pp + r * 128, dsc + r * kTileRows, 0, b, cr, accd[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < NRT; ++i) {
+          const int r = warp + kDecWarps * i;
+          if (r < ntiles)
+            group_mma<BITS>(pp + r * 128, pp + 8 * d + r * 64, dsc + r * kTileRows, 0, b, accd[i]);
+        }
       }
     }
     __syncthreads();
@@ -605,21 +595,29 @@ __global__ void __maxnreg__(88)
       refill(pg + 3);   // the Wd slot is free
     }
   }
-  if (j < my && tid == 0) {
-    // a wait ran out: let every requested piece land before the CTA exits
-    for (int p = 3 * j; p < issued; ++p) mbar_wait(&full[p % nslots], (p / nslots) & 1, ctl, 0x605);
+  if (tid == 0) {
+    // a wait ran out: let every requested copy land before the CTA exits
+    if (j < my)
+      for (int p = 3 * j; p < issued; ++p) mbar_wait(&full[p % nslots], (p / nslots) & 1, ctl, 0x605);
+    if (!ok) mbar_wait(&xbar, 0, ctl, 0x606);
   }
   // this CTA's partial sums: lane (g, t) of tile r holds rows g, g+8 and tokens 2t, 2t+1
   if (my > 0) {
     const int g = lane >> 2, t = lane & 3;
+    float* p0 = partial + ((size_t)blockIdx.x * T + 2 * t) * d + warp * kTileRows + g;
+    float* p1 = p0 + d;
+    const bool w0 = 2 * t < T, w1 = 2 * t + 1 < T;
 #pragma unroll
     for (int i = 0; i < NRT; ++i) {
-      const int r = warp + kDecWarps * i;
-      if (r >= ntiles) continue;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int n = 2 * t + (e & 1), row = r * kTileRows + g + 8 * (e >> 1);
-        if (n < T) partial[((size_t)blockIdx.x * T + n) * d + row] = accd[i][e];
+      if (warp + kDecWarps * i >= ntiles) break;
+      const int o = i * kDecWarps * kTileRows;
+      if (w0) {
+        p0[o] = accd[i][0];
+        p0[o + 8] = accd[i][2];
+      }
+      if (w1) {
+        p1[o] = accd[i][1];
+        p1[o + 8] = accd[i][3];
       }
     }
   }
@@ -809,7 +807,7 @@ int decode_grid() {
 }
 
 template <int BITS, int NRT>
-static cudaError_t launch_expert(const DecMaps& mp, const LayerDev& L, const uint16_t* x, int T,
+static cudaError_t launch_expert(const DecMaps& mp, const LayerDev& L, const unsigned char* xfrag, int T,
                                  const float* logits, const int32_t* ids, const float* w,
                                  int32_t* ids_out, float* w_out, float* partial, uint32_t flags,
                                  Control* ctl, int nslots, cudaStream_t st) {
@@ -818,7 +816,7 @@ static cudaError_t launch_expert(const DecMaps& mp, const LayerDev& L, const uin
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)m.total);
   if (e != cudaSuccess) return e;
   return launch_pdl(decode_expert_kernel<BITS, NRT>, dim3(decode_grid()), dim3(kDecWarps * 32),
-                    m.total, st, mp, L, x, T, logits, ids, w, ids_out, w_out, partial, flags, ctl,
+                    m.total, st, mp, L, xfrag, T, logits, ids, w, ids_out, w_out, partial, flags, ctl,
                     nslots);
 }
 
@@ -828,6 +826,7 @@ cudaError_t launch_decode(const LayerDev& L, const uint16_t* x, int T, const flo
                           cudaStream_t st) {
   Control* ctl = reinterpret_cast<Control*>(ws + lay.ctl);
   float* partial = reinterpret_cast<float*>(ws + lay.partial);
+  const unsigned char* xf = reinterpret_cast<const unsigned char*>(ws + lay.xfrag);
   const int nslots = dec_nslots(L.d, L.E, L.bits);
   if (nslots < 2) return cudaErrorInvalidValue;
   DecMaps mp;
@@ -835,15 +834,19 @@ cudaError_t launch_decode(const LayerDev& L, const uint16_t* x, int T, const flo
   cudaError_t e;
   const bool wide = L.d / kTileRows > kDecWarps * 8;
   if (L.bits == 2)
-    e = wide ? launch_expert<2, 16>(mp, L, x, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st)
-             : launch_expert<2, 8>(mp, L, x, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st);
+    e = wide ? launch_expert<2, 16>(mp, L, xf, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st)
+             : launch_expert<2, 8>(mp, L, xf, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st);
   else
-    e = wide ? launch_expert<3, 16>(mp, L, x, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st)
-             : launch_expert<3, 8>(mp, L, x, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st);
+    e = wide ? launch_expert<3, 16>(mp, L, xf, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st)
+             : launch_expert<3, 8>(mp, L, xf, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st);
   if (e != cudaSuccess) return e;
   return launch_pdl(decode_combine_kernel, dim3(L.d / kCombRows), dim3(kCombThreads), 0, st,
                     static_cast<const float*>(partial), x, y, T, L.d, flags,
                     static_cast<const Control*>(ctl));
+}
+
+size_t decode_xfrag_bytes(const LayerDev& L) {
+  return (size_t)(L.d / kGroup) * (32 * 16 + kMaxDecodeT * 4);
 }
 
 size_t decode_partial_bytes(const LayerDev& L, int T) {

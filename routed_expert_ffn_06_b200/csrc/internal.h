@@ -36,6 +36,7 @@ struct WsLayout {
   size_t ids;        // int32 [T][k]
   size_t w;          // fp32 [T][k]
   size_t partial;    // decode: fp32 partial sums [expert CTAs][T][d]
+  size_t xfrag;      // decode: token operands of the expert kernel (B fragments, corrections)
   size_t xn;         // prefill: bf16 [T][d] (PRENORM)
   size_t x16;        // prefill: fp16 [T][d]
   size_t counts;     // prefill: int32 [E+1]
@@ -53,9 +54,12 @@ struct WsLayout {
 WsLayout ws_layout(const LayerDev& L, int T);
 
 // launchers (return cudaError_t of the launch)
-// Router logits for a decode window (T <= 8): one warp per expert row.
+// Router logits for a decode window (T <= 8): one warp per expert row; with
+// xfrag non-null it also writes the expert kernel's token operands there
+// (logits may be null: operands only).
 cudaError_t launch_router_gemv(const LayerDev& L, const uint16_t* x, int T, uint32_t flags,
-                               float* logits, Control* ctl, cudaStream_t st);
+                               float* logits, unsigned char* xfrag, Control* ctl,
+                               cudaStream_t st);
 // Top-k selection and renormalised weights, one warp per token.
 cudaError_t launch_topk(const LayerDev& L, const float* logits, int T, int32_t* ids, float* w,
                         uint32_t flags, Control* ctl, cudaStream_t st);
@@ -69,6 +73,7 @@ cudaError_t launch_router_tc(const LayerDev& L, const uint16_t* x, int T, float*
 constexpr int kMaxDecodeCtas = 160;
 bool decode_fits(int d, int E, int Fmax, int bits, int T);
 size_t decode_partial_bytes(const LayerDev& L, int T);
+size_t decode_xfrag_bytes(const LayerDev& L);
 // Decode expert step + combine.  Routing from `logits` (selected in the
 // kernel; ids_out / w_out receive it when non-null) or given (`ids`, `w`).
 cudaError_t launch_decode(const LayerDev& L, const uint16_t* x, int T, const float* logits,

@@ -126,6 +126,8 @@ WsLayout ws_layout(const LayerDev& L, int T) {
   o += align256(Tn * L.k * sizeof(float));
   w.partial = o;
   o += align256(decode_partial_bytes(L, T));
+  w.xfrag = o;
+  o += align256(decode_xfrag_bytes(L));
   w.decode_total = o;   // the decode path (router for T <= 8, decode step) uses no more
   if (T > 0) {
     size_t parts[16];
@@ -196,7 +198,8 @@ moe_status block_forward(const moe_layer* layer, const void* x_bf16, int32_t T, 
     Control* ctl = reinterpret_cast<Control*>(w + lay.ctl);
     float* logits = reinterpret_cast<float*>(w + lay.logits);
     const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-    cudaError_t e = launch_router_gemv(L, x, T, flags, logits, ctl, st);
+    cudaError_t e = launch_router_gemv(L, x, T, flags, logits,
+                                       reinterpret_cast<unsigned char*>(w + lay.xfrag), ctl, st);
     if (e == cudaSuccess)
       e = launch_decode(L, x, T, logits, nullptr, nullptr, ids, wt, static_cast<uint16_t*>(y_bf16),
                         flags, w, lay, st);
@@ -259,7 +262,7 @@ moe_status moe_route_topk(const moe_layer* layer, const void* x_bf16, int32_t T,
   float* logits = logits_or_null ? logits_or_null : reinterpret_cast<float*>(w + lay.logits);
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
   if (T <= kMaxDecodeT) {
-    cudaError_t e = launch_router_gemv(L, x, T, flags, logits, ctl, st);
+    cudaError_t e = launch_router_gemv(L, x, T, flags, logits, nullptr, ctl, st);
     if (e == cudaSuccess) e = launch_topk(L, logits, T, topk_ids, topk_w, flags, ctl, st);
     return from_cuda(e);
   }
@@ -292,9 +295,17 @@ moe_status moe_expert_ffn_decode(const moe_layer* layer, const void* x_bf16, int
   if (y_bf16 == x_bf16) return MOE_ERR_INVALID_ARG;
   if ((s = check_device()) != MOE_OK) return s;
   if (T == 0) return MOE_OK;
-  return from_cuda(launch_decode(L, static_cast<const uint16_t*>(x_bf16), T, nullptr, topk_ids,
-                                 topk_w, nullptr, nullptr, static_cast<uint16_t*>(y_bf16), flags,
-                                 static_cast<char*>(ws), lay, static_cast<cudaStream_t>(stream)));
+  // the token operands of the expert kernel, then the expert step
+  char* w = static_cast<char*>(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  cudaError_t e = launch_router_gemv(L, x, T, flags, nullptr,
+                                     reinterpret_cast<unsigned char*>(w + lay.xfrag),
+                                     reinterpret_cast<Control*>(w + lay.ctl), st);
+  if (e == cudaSuccess)
+    e = launch_decode(L, x, T, nullptr, topk_ids, topk_w, nullptr, nullptr,
+                      static_cast<uint16_t*>(y_bf16), flags, w, lay, st);
+  return from_cuda(e);
 }
 
 moe_status moe_expert_ffn_prefill(const moe_layer* layer, const void* x_bf16, int32_t T,

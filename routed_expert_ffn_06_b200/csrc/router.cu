@@ -30,11 +30,12 @@ namespace moe {
 constexpr int kGemvWarps = 4;
 template <int NPRE>
 __global__ void __maxnreg__(88) router_gemv_kernel(
-    LayerDev L, const uint16_t* __restrict__ x, int T, uint32_t flags, float* __restrict__ logits) {
+    const __grid_constant__ LayerDev L, const uint16_t* __restrict__ x, int T, uint32_t flags, float* __restrict__ logits,
+    unsigned char* __restrict__ xfrag, Control* ctl) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * kGemvWarps + warp;
   const int d = L.d, nc4 = d / 4;
-  const bool have = e < L.E;
+  const bool have = logits != nullptr && e < L.E;
   const float4* wr = reinterpret_cast<const float4*>(L.Wr + (size_t)(have ? e : 0) * d);
   float4 w[NPRE];
 #pragma unroll
@@ -46,75 +47,121 @@ __global__ void __maxnreg__(88) router_gemv_kernel(
   // let the next grid (which reads x before its own wait) start only then
   pdl_wait();
   pdl_launch_dependents();
-  if (!have) return;
   const bool pn = flags & MOE_F_PRENORM;
-  float inv[kMaxDecodeT];
+  // 1 / RMS of token t (the sum of squares in the expert kernel's fixed order)
+  auto inv_rms = [&](int t) {
+    float ss = 0.f;
+#pragma unroll 1
+    for (int i = lane * 8; i < d; i += 256) {
+      const uint4 v = *reinterpret_cast<const uint4*>(x + (size_t)t * d + i);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int t = 0; t < kMaxDecodeT; ++t) {
-    inv[t] = 1.f;
-    if (pn && t < T) {
-      float ss = 0.f;
-      for (int i = lane * 8; i < d; i += 256) {
-        const uint4 v = *reinterpret_cast<const uint4*>(x + (size_t)t * d + i);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float a = __uint_as_float(w4[q] << 16), b = __uint_as_float(w4[q] & 0xFFFF0000u);
-          ss += a * a + b * b;
-        }
+      for (int q = 0; q < 4; ++q) {
+        const float a = __uint_as_float(w4[q] << 16), b = __uint_as_float(w4[q] & 0xFFFF0000u);
+        ss += a * a + b * b;
       }
-      ss = warp_sum(ss);
-      inv[t] = rsqrtf(ss / (float)d + kRmsEps);
     }
-  }
-  auto xval = [&](int t, int c, float (&v)[4]) {   // x[t][4c .. 4c+3], normalised when asked
-    const uint2 u = *reinterpret_cast<const uint2*>(x + (size_t)t * d + 4 * c);
-    v[0] = __uint_as_float(u.x << 16);
-    v[1] = __uint_as_float(u.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(u.y << 16);
-    v[3] = __uint_as_float(u.y & 0xFFFF0000u);
-    if (pn) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) v[q] = __bfloat162float(__float2bfloat16_rn(v[q] * inv[t]));
-    }
+    return rsqrtf(warp_sum(ss) / (float)d + kRmsEps);
   };
+  // The expert kernel's operands for the window's tokens: per (quantisation
+  // group c, token n) the 32 values as the mma B fragments of lanes 4n..4n+3
+  // (fp16; 2-bit: value / 4^m for columns 8m..8m+7, the offset form) and, for
+  // 2-bit, the correction sum of B * (1024 + 2 * 4^m).  One warp per (c, n),
+  // lane q < 16 holding columns 2q, 2q+1.  fp16 operands: values outside the
+  // fp16 range are flagged (always on).
+  if (xfrag) {
+    const int nG = d / kGroup, npairs = kMaxDecodeT * nG;
+    uint32_t* xs = reinterpret_cast<uint32_t*>(xfrag);
+    float* corr = reinterpret_cast<float*>(xfrag + (size_t)nG * 32 * 16);
+    bool bad = false;
+#pragma unroll 1
+    for (int p = blockIdx.x * kGemvWarps + warp; p < npairs; p += gridDim.x * kGemvWarps) {
+      const int c = p >> 3, n = p & 7, m = (lane >> 2) & 3;
+      const float inv = (pn && n < T) ? inv_rms(n) : 1.f;
+      float v0 = 0.f, v1 = 0.f;
+      if (lane < 16 && n < T) {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(x + (size_t)n * d + 32 * c + 2 * lane);
+        v0 = __uint_as_float(u << 16);
+        v1 = __uint_as_float(u & 0xFFFF0000u);
+        if (pn) {
+          v0 = __bfloat162float(__float2bfloat16_rn(v0 * inv));
+          v1 = __bfloat162float(__float2bfloat16_rn(v1 * inv));
+        }
+        bad |= !(fabsf(v0) <= 65504.f) || !(fabsf(v1) <= 65504.f);
+      }
+      float cs = 0.f;
+      __half2 bh;
+      if (L.bits == 2) {
+        const float sc = 1.f / (float)(1 << (2 * m));
+        bh = __floats2half2_rn(v0 * sc, v1 * sc);
+        cs = (__low2float(bh) + __high2float(bh)) * (1024.f + 2.f * (float)(1 << (2 * m)));
+      } else {
+        bh = __floats2half2_rn(v0, v1);
+      }
+      if (lane < 16) xs[((size_t)(c * 32 + n * 4 + (lane & 3))) * 4 + m] = h2_as_u32(bh);
+      cs = warp_sum(lane < 16 ? cs : 0.f);
+      if (lane == 0) corr[c * kMaxDecodeT + n] = cs;
+    }
+    if (bad) record_error(ctl, kErrNonFinite, 0x120);
+  }
+  if (!have) return;
   const float b = L.bias ? L.bias[e] : 0.f;
+  // two tokens per pass: twice the loads in flight per memory round trip
+#pragma unroll 1
+  for (int t = 0; t < T; t += 2) {
+    const bool two = t + 1 < T;
+    const float inv0 = pn ? inv_rms(t) : 1.f;
+    const float inv1 = (pn && two) ? inv_rms(t + 1) : 1.f;
+    const uint16_t* x0 = x + (size_t)t * d;
+    const uint16_t* x1 = two ? x0 + d : x0;
+    auto dot4 = [&](float acc, const float4& wv, const uint16_t* xt, float inv, int c) {
+      const uint2 u = *reinterpret_cast<const uint2*>(xt + 4 * c);
+      float v[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                    __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
+      if (pn) {
 #pragma unroll
-  for (int t = 0; t < kMaxDecodeT; ++t) {
-    if (t >= T) break;
-    float acc = 0.f;
+        for (int q = 0; q < 4; ++q) v[q] = __bfloat162float(__float2bfloat16_rn(v[q] * inv));
+      }
+      acc = fmaf(v[0], wv.x, acc);
+      acc = fmaf(v[1], wv.y, acc);
+      acc = fmaf(v[2], wv.z, acc);
+      return fmaf(v[3], wv.w, acc);
+    };
+    float a0 = 0.f, a1 = 0.f;
 #pragma unroll
     for (int j = 0; j < NPRE; ++j) {
       const int c = lane + 32 * j;
       if (c < nc4) {
-        float v[4];
-        xval(t, c, v);
-        acc = fmaf(v[0], w[j].x, acc);
-        acc = fmaf(v[1], w[j].y, acc);
-        acc = fmaf(v[2], w[j].z, acc);
-        acc = fmaf(v[3], w[j].w, acc);
+        a0 = dot4(a0, w[j], x0, inv0, c);
+        a1 = dot4(a1, w[j], x1, inv1, c);
       }
     }
-    for (int c = lane + 32 * NPRE; c < nc4; c += 32) {   // rows longer than the prefetch
+#pragma unroll 1
+    for (int c = lane + 32 * NPRE; c < nc4; c += 32) {
       const float4 wv = ldg_nc_f4(wr + c);
-      float v[4];
-      xval(t, c, v);
-      acc = fmaf(v[0], wv.x, acc);
-      acc = fmaf(v[1], wv.y, acc);
-      acc = fmaf(v[2], wv.z, acc);
-      acc = fmaf(v[3], wv.w, acc);
+      a0 = dot4(a0, wv, x0, inv0, c);
+      a1 = dot4(a1, wv, x1, inv1, c);
     }
-    acc = warp_sum(acc);
-    if (lane == 0) logits[(size_t)t * L.E + e] = acc + b;
+    a0 = warp_sum(a0);
+    a1 = warp_sum(a1);
+    if (lane == 0) {
+      logits[(size_t)t * L.E + e] = a0 + b;
+      if (two) logits[(size_t)(t + 1) * L.E + e] = a1 + b;
+    }
   }
 }
 
 cudaError_t launch_router_gemv(const LayerDev& L, const uint16_t* x, int T, uint32_t flags,
-                               float* logits, Control* ctl, cudaStream_t st) {
-  (void)ctl;
-  const dim3 grid((L.E + kGemvWarps - 1) / kGemvWarps);
+                               float* logits, unsigned char* xfrag, Control* ctl,
+                               cudaStream_t st) {
+  // logits: one warp per expert row; token fragments only: enough warps for
+  // the (group, token) pairs
+  const int rows = logits ? L.E : 0;
+  const int pairs = xfrag ? kMaxDecodeT * (L.d / kGroup) : 0;
+  const int warps = rows > pairs ? rows : pairs;
+  const dim3 grid((warps + kGemvWarps - 1) / kGemvWarps);
   return launch_pdl(router_gemv_kernel<16>, grid, dim3(kGemvWarps * 32), 0, st, L, x, T, flags,
-                    logits);
+                    logits, xfrag, ctl);
 }
 
 // ------------------------------------------------------------ prefill router
