@@ -60,6 +60,12 @@
  *    bits in {2, 3}; group == 32.
  *  - Alignment: x, y, codes, scales, shared_codes, shared_scales, router_w:
  *    16 bytes.
+ *  - Precision: the expert products take fp16 operands.  Token values (after
+ *    the optional RMSNorm) above 65,504 in magnitude saturate, and the kernels
+ *    report them in the error word (kErrNonFinite, always checked); values
+ *    below 6.1e-5 in magnitude keep only fp16-subnormal precision.  Routing
+ *    logits are fp32; the output is accumulated in fp32 and rounded once to
+ *    bf16.
  */
 #ifndef MOE_H
 #define MOE_H
@@ -166,9 +172,8 @@ moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t
                              uint32_t flags, void* ws, size_t ws_bytes, void* stream);
 
 /* moe_block_forward for a decode window (0 <= T <= 4) without a caller
- * workspace: the scratch is an 8 MiB array in the library's device memory, one
- * per device (a T = 4 window of a d = 2048, 512-expert layer needs about
- * 5.3 MB).  The Strata pages have no counterpart; this is for callers that
+ * workspace: the scratch is a 2 MiB array in the library's device memory, one
+ * per device.  The Strata pages have no counterpart; this is for callers that
  * cannot allocate or own a workspace (a plain C host without a device
  * allocator, a step loop that must not call cudaMalloc, which synchronises the
  * device).
@@ -184,9 +189,11 @@ moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t
  *    workspace to inspect them.
  *  - One scratch per device: calls on the same device must be ordered (one
  *    stream, or events); calls that overlap on the GPU race on the scratch.
- *  - Shapes whose decode workspace exceeds 8 MiB return
- *    MOE_ERR_WORKSPACE_TOO_SMALL; T > 4 returns MOE_ERR_UNSUPPORTED_SHAPE;
- *    both before anything is enqueued.
+ *  - Shapes whose workspace (moe_workspace_bytes(layer, T)) exceeds 2 MiB
+ *    return MOE_ERR_WORKSPACE_TOO_SMALL; T > 4 returns
+ *    MOE_ERR_UNSUPPORTED_SHAPE; both before anything is enqueued.  A layer
+ *    too wide for the decode kernels (see moe_expert_ffn_decode) takes the
+ *    prefill step, whose full workspace must then fit in the 2 MiB.
  *  - Status codes match moe_block_forward's (MOE_ERR_NO_DEVICE without a
  *    current sm_100 device). */
 moe_status moe_block_forward_noalloc(const moe_layer* layer, const void* x_bf16, int32_t T,

@@ -24,7 +24,7 @@ constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
 // Workspace control block (first 256 bytes of every workspace).
 struct Control {
   uint32_t err;            // OR of kErr* bits
-  uint32_t decode_ctas;    // expert CTAs of the last decode call holding partial sums
+  uint32_t router_done;    // CTAs of the small-T router that finished (self-resetting)
   uint32_t prefill_done;   // CTAs of the prefill bucketing pass that finished (self-resetting)
   uint32_t pad0;
   uint32_t err_where;      // first failing site (debug aid)
@@ -158,16 +158,6 @@ __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
 
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
-
-// 16-byte read-only load that does not allocate in L1 (constant weights read
-// once per CTA).
-__device__ __forceinline__ float4 ldg_nc_f4(const void* p) {
-  float4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "l"(p));
-  return v;
-}
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);

@@ -6,43 +6,32 @@
 // check").  So the window's selected experts are deduplicated and every
 // selected expert's packed weights are streamed from HBM exactly once per call.
 //
-// Split-K over the expert's hidden dimension.  A work unit is one 32-row slice
-// s of one expert u: rows 32s..32s+31 of Wg and Wu (two packed 16-row tiles
-// each) and the matching 32-column group of Wd (one quantisation group of every
-// output row).  A CTA computes the slice's gate/up products, applies SwiGLU
-// and the routing weight, and multiplies the 32 hidden values of each token
-// with its Wd columns: the hidden vector never leaves the SM.  Each CTA adds
-// its units' contributions to all d outputs in registers and writes one fp32
-// partial sum per token and output; a small combine kernel adds the CTAs'
-// partial sums in CTA order (deterministic, no atomics), adds the residual and
-// rounds once to bf16.
-//
-// One unit arrives as three equal pieces of d*(code bytes per group + 2) bytes
-// each: the Wg slice and the Wu slice (two bulk copies each: codes and scales,
-// contiguous in the packed layout) and the Wd group column (strided across the
-// output-row tiles: one 4-D TMA load per plane).  Pieces stream through a ring
-// of shared-memory slots with one mbarrier each; one thread issues them in the
-// order they are consumed.
-//
-// Kernels of a window, chained with programmatic dependent launch (PDL):
-//   router (router.cu) -> decode_expert_kernel -> decode_combine_kernel.
-// decode_expert_kernel selects the window's top-k itself from the router's
-// fp32 logits (every CTA, redundantly: no extra launch and no serial tail)
-// and deduplicates the selections; the shared expert's units are requested
-// before the kernel waits for the router, since they do not depend on it.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
+// Two kernels, chained with programmatic dependent launch (PDL):
+//  * decode_gu: work item = (expert u, 16-row tile of Wg and Wu).  A quad of
+//    four warps shares an item: each warp takes pieces of 16 quantisation
+//    groups of the K = d contraction, streams them into its own shared-memory
+//    stages with warp-wide cp.async, dequantises the 2/3-bit codes straight into
+//    mma.sync A fragments (LOP3 + HFMA2: no shared-memory round trip for the
+//    fp16 weights) and multiplies them with the window's tokens (B fragments;
+//    n = 8 covers T <= 8).  The quad adds its partial sums through shared
+//    memory, applies SwiGLU and the routing weight and writes
+//    hw[u][f][t] = w_u[t] * silu(g) * up  (fp16, in B-fragment order).
+//  * decode_dn: one CTA per 16-row tile of the output.  Its Wd tiles depend
+//    only on the routing, so they are requested before the kernel waits for
+//    decode_gu; the hidden vectors follow after the wait.  Warps sum over the
+//    experts, then the CTA adds the warps in a fixed order (deterministic, no
+//    atomics) and writes y (bf16, optional residual).
+// The shared expert is expert u = 0 with weight 1 for every token.
+// Each warp owns its stages and fills them itself (gate/up: cp.async groups;
+// down: bulk copies on per-stage mbarriers, every wait on the current phase).
 #include "internal.h"
-#include "select.cuh"
 #include "tc.cuh"
 
 namespace moe {
 
 constexpr int kMaxExp = kMaxDecodeT * 16 + 1;   // window entries + shared
-constexpr int kDecWarps = 16;
+constexpr int kGuWarps = 16;                 // four quads
+constexpr int kDnWarps = 16;
 
 struct ExpList {
   int n;                       // experts in the list (shared first when present)
@@ -57,7 +46,6 @@ struct ExpList {
 // are replaced by 0 and flagged, so no later address leaves the expert array.
 __device__ void expert_list_prologue(const LayerDev& L, ExpList* s, int* slot_s, int* first,
                                      Control* ctl) {
-#pragma unroll 1
   for (int e = threadIdx.x; e < L.E; e += blockDim.x) {
     int sl = L.slot[e];
     if (sl < 0 || sl >= L.E) {
@@ -67,7 +55,6 @@ __device__ void expert_list_prologue(const LayerDev& L, ExpList* s, int* slot_s,
     slot_s[e] = sl;
     first[e] = 0x7FFFFFFF;
   }
-#pragma unroll 1
   for (int i = threadIdx.x; i < kMaxExp * kMaxDecodeT; i += blockDim.x) (&s->w[0][0])[i] = 0.f;
 }
 
@@ -244,39 +231,325 @@ __device__ __forceinline__ void group_mma_2b_offset(const unsigned char* lo, con
   acc[3] = fmaf(s1, tmp[3], acc[3]);
 }
 
-
-// ------------------------------------------------------------- tensor maps
-// The down projection's 32-column group s of every 16-row output tile, for
-// one slot: 4-D views of the packed Wd bytes (see dec_maps()).
-struct alignas(64) DecMaps {
-  CUtensorMap lo, hi, sc;      // routed experts (slot dimension = n_experts)
-  CUtensorMap slo, shi, ssc;   // shared expert (slot dimension = 1)
+// Source of expert u (shared when u == 0 and the layer has one).
+struct ExpSrc {
+  const uint8_t* codes;
+  const uint16_t* scales;
+  int F;
 };
-
-__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1,
-                                            int c2, int c3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
-      : "memory");
+__device__ __forceinline__ ExpSrc expert_src(const LayerDev& L, const ExpList* s, int u,
+                                             Control* ctl) {
+  ExpSrc r;
+  (void)ctl;
+  if (s->id[u] < 0) {
+    r.codes = L.scodes;
+    r.scales = L.sscales;
+    r.F = L.Fs;
+  } else {
+    const int slot = s->slot[u];
+    r.codes = L.codes + (long long)slot * L.cbe;
+    r.scales = L.scales + (long long)slot * L.nse;
+    r.F = L.F;
+  }
+  return r;
 }
 
-// ------------------------------------------------------------ smem layout
-// piece: bytes of one Wg slice, one Wu slice or one Wd group column (equal).
-__host__ __device__ inline uint32_t dec_piece_bytes(int d, int bits) {
-  return (uint32_t)d * (uint32_t)(group_bytes(bits) + 2);
-}
-struct DecSmem {
-  size_t bars, list, first, sel, xs, corr, part, hfrag, slots, total;
-  size_t slot;   // slot stride (a piece, rounded up to 128 bytes)
+// ------------------------------------------------------------------ gate/up
+// hw layout (fp16): [u][c = f/32][lane < 4T][8 halves] -- the B fragments of
+// the down projection for the T real tokens, so a CTA can bulk-copy one
+// expert's hidden vector (2*F*T bytes) in one piece.
+__host__ __device__ inline size_t hw_expert_halves(int Fmax, int T) { return (size_t)Fmax * T; }
+
+constexpr int kGuPiece = 16;                 // groups per piece of a gate/up item
+struct GuSmem {
+  size_t bars, list, first, xs, corr, part, stages, total, stage_bytes;
+  int spw;                                   // stages per warp
 };
-__host__ __device__ inline DecSmem dec_smem(int d, int E, int bits, int nslots) {
-  DecSmem m;
+__host__ __device__ inline size_t gu_stage_bytes(int bits) {
+  // Wg lo | Wg hi | Wu lo | Wu hi | Wg scales | Wu scales   (one piece)
+  const size_t lo = kGuPiece * kTileRows * 8, hi = bits == 3 ? kGuPiece * kTileRows * 4 : 0;
+  return 2 * (lo + hi) + 2 * kGuPiece * kTileRows * 2;
+}
+__host__ __device__ inline GuSmem gu_smem(int d, int E, int bits, int spw) {
+  GuSmem m;
   const int nG = d / kGroup;
   size_t o = 0;
+  m.spw = spw;
   m.bars = o;
-  o += (size_t)nslots * sizeof(uint64_t);
+  o += (size_t)kGuWarps * spw * sizeof(uint64_t);
+  o = (o + 15) & ~size_t(15);
+  m.list = o;
+  o += sizeof(ExpList);
+  o = (o + 15) & ~size_t(15);
+  m.first = o;
+  o += 2 * (size_t)E * sizeof(int);   // first-occurrence scratch, slot table
+  o = (o + 127) & ~size_t(127);
+  m.xs = o;
+  o += (size_t)nG * 32 * 16;
+  m.corr = o;                                // [group][token] fp32 (2-bit offset form)
+  o += (size_t)nG * kMaxDecodeT * sizeof(float);
+  m.part = o;                                // [quad][2][warp in quad][lane][8] floats
+  o += (size_t)(kGuWarps / 4) * 2 * 4 * 32 * 8 * sizeof(float);
+  o = (o + 127) & ~size_t(127);
+  m.stages = o;
+  m.stage_bytes = gu_stage_bytes(bits);
+  o += (size_t)kGuWarps * spw * m.stage_bytes;
+  m.total = o;
+  return m;
+}
+
+__device__ __forceinline__ void gu_item(const LayerDev& L, int i, int Fs16, int F16, int* u,
+                                        int* tile) {
+  if (i < Fs16) {
+    *u = 0;
+    *tile = i;
+  } else {
+    *u = (L.Fs > 0 ? 1 : 0) + (i - Fs16) / F16;
+    *tile = (i - Fs16) % F16;
+  }
+}
+
+// Warp-wide copy of `bytes` (a multiple of 16, both ends 16-byte aligned) from
+// global to shared memory, 16 bytes per lane and instruction (cp.async: many
+// small pieces in flight without going through the bulk-copy unit).
+__device__ __forceinline__ void warp_cp_async(void* dst, const void* src, uint32_t bytes) {
+  const int lane = threadIdx.x & 31;
+  for (uint32_t o = (uint32_t)lane * 16; o < bytes; o += 512)
+    cp_async16(static_cast<unsigned char*>(dst) + o, static_cast<const unsigned char*>(src) + o, 16);
+}
+// Wait until at most n of this thread's cp.async groups are pending (n <= 3).
+__device__ __forceinline__ void cp_async_wait_upto(int n) {
+  if (n <= 0)
+    cp_async_wait<0>();
+  else if (n == 1)
+    cp_async_wait<1>();
+  else if (n == 2)
+    cp_async_wait<2>();
+  else
+    cp_async_wait<3>();
+}
+
+// Piece p (groups kGuPiece*p onwards) of gate/up item (u, tile) into a stage, by
+// the whole warp: one cp.async group.
+template <int BITS>
+__device__ __forceinline__ void gu_copy(const LayerDev& L, const ExpList* list, int u, int tile,
+                                        int p, unsigned char* st, Control* ctl) {
+  const int d = L.d, nG = d / kGroup;
+  const int g0 = kGuPiece * p, np = min(kGuPiece, nG - g0);
+  const ExpSrc src = expert_src(L, list, u, ctl);
+  const long long tcb = (long long)nG * kTileRows * group_bytes(BITS);
+  const long long mcb = mat_codes_bytes(src.F, d, BITS);
+  const long long msc = (long long)src.F * nG;
+  const uint32_t blo = np * kTileRows * 8, bhi = BITS == 3 ? np * kTileRows * 4 : 0;
+  const uint32_t bsc = np * kTileRows * 2;
+  const size_t LO = kGuPiece * kTileRows * 8, HI = BITS == 3 ? kGuPiece * kTileRows * 4 : 0;
+#pragma unroll
+  for (int mat = 0; mat < 2; ++mat) {
+    const uint8_t* tb = src.codes + (mat ? mcb : 0) + tile * tcb;
+    unsigned char* so = st + mat * (LO + HI);
+    warp_cp_async(so, tb + g0 * kTileRows * 8, blo);
+    if (BITS == 3) warp_cp_async(so + LO, tb + (long long)nG * kTileRows * 8 + g0 * kTileRows * 4, bhi);
+    const uint16_t* sb = src.scales + (mat ? msc : 0) + (long long)tile * kTileRows * nG;
+    warp_cp_async(st + 2 * (LO + HI) + mat * kGuPiece * kTileRows * 2, sb + g0 * kTileRows, bsc);
+  }
+  cp_async_commit();
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kGuWarps * 32, 1)
+    decode_gu_kernel(LayerDev L, const uint16_t* __restrict__ x, int T,
+                     const int32_t* __restrict__ ids, const float* __restrict__ wts,
+                     __half* __restrict__ hw, int Fmax, uint32_t flags, Control* ctl, int spw) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const GuSmem m = gu_smem(L.d, L.E, BITS, spw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + m.bars);
+  ExpList* list = reinterpret_cast<ExpList*>(smem + m.list);
+  int* first = reinterpret_cast<int*>(smem + m.first);
+  uint4* xs = reinterpret_cast<uint4*>(smem + m.xs);
+  float* corr = reinterpret_cast<float*>(smem + m.corr);
+  float* part = reinterpret_cast<float*>(smem + m.part);
+  __shared__ float inv_rms[kMaxDecodeT];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nthreads = kGuWarps * 32;
+  const int d = L.d, nG = d / kGroup;
+  if (tid == 0) {
+    for (int s = 0; s < kGuWarps * spw; ++s) mbar_init(&bars[s], 1);
+    fence_barrier_init();
+  }
+  expert_list_prologue(L, list, first + L.E, first, ctl);
+  // ---- tokens -> B fragments.  x is an input of the whole block: readable
+  //      before this grid waits on the router.
+  if (warp < T && (flags & MOE_F_PRENORM)) {
+    float ss = 0.f;
+#pragma unroll 4
+    for (int i = lane * 8; i < d; i += 256) {
+      const uint4 v = *reinterpret_cast<const uint4*>(x + (size_t)warp * d + i);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float a = __uint_as_float(w4[j] << 16), b = __uint_as_float(w4[j] & 0xFFFF0000u);
+        ss += a * a + b * b;
+      }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) inv_rms[warp] = rsqrtf(ss / (float)d + 1e-6f);
+  }
+  __syncthreads();
+  // one (token n, group c) pair per thread: 32 values -> the 16-byte B
+  // fragments of lanes 4n .. 4n+3 (pair m of lane 4n+t = columns 8m+2t, +1)
+  for (int pidx = tid; pidx < kMaxDecodeT * nG; pidx += nthreads) {
+    const int c = pidx >> 3, n = pidx & 7;
+    uint4 out[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                    make_uint4(0, 0, 0, 0)};
+    if (n < T) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)n * d + 32 * c);
+      uint32_t w[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = src[q];
+        w[4 * q] = v.x;
+        w[4 * q + 1] = v.y;
+        w[4 * q + 2] = v.z;
+        w[4 * q + 3] = v.w;
+      }
+      const bool pn = flags & MOE_F_PRENORM;
+      const float sc = pn ? inv_rms[n] : 1.f;
+      uint32_t h2[16];
+      float cs = 0.f;
+      bool bad = false;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {   // w[q] holds columns 2q, 2q+1 = 8m + 2t (+1), q = 4m + t
+        float v0 = __uint_as_float(w[q] << 16), v1 = __uint_as_float(w[q] & 0xFFFF0000u);
+        if (pn) {
+          v0 = __bfloat162float(__float2bfloat16_rn(v0 * sc));
+          v1 = __bfloat162float(__float2bfloat16_rn(v1 * sc));
+        }
+        // fp16 operands: values outside the fp16 range are flagged (always on)
+        bad |= !(fabsf(v0) <= 65504.f) || !(fabsf(v1) <= 65504.f);
+        if (BITS == 2) {
+          // offset form: B = x / 4^m; correction sum B * (1024 + 2 * 4^m)
+          const float inv = 1.f / (float)(1 << (2 * (q >> 2)));
+          const __half2 bh = __floats2half2_rn(v0 * inv, v1 * inv);
+          h2[q] = h2_as_u32(bh);
+          cs += (__low2float(bh) + __high2float(bh)) * (1024.f + 2.f * (float)(1 << (2 * (q >> 2))));
+        } else {
+          h2[q] = h2_as_u32(__floats2half2_rn(v0, v1));
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) out[t] = make_uint4(h2[t], h2[4 + t], h2[8 + t], h2[12 + t]);
+      corr[c * kMaxDecodeT + n] = cs;
+      if (bad) record_error(ctl, kErrNonFinite, 0x400);
+    } else {
+      corr[c * kMaxDecodeT + n] = 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) xs[c * 32 + n * 4 + t] = out[t];
+  }
+  __syncthreads();
+  pdl_wait();
+  pdl_launch_dependents();
+  if (warp == 0) build_expert_list(ids, wts, T, L, list, first + L.E, first, ctl);
+  __syncthreads();
+
+  const int Fs16 = L.Fs / kTileRows, F16 = L.F / kTileRows;
+  const int n_items = Fs16 + (list->n - (L.Fs > 0 ? 1 : 0)) * F16;
+  const int my_items = n_items > (int)blockIdx.x ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int quad = warp >> 2, wq = warp & 3, nquads = kGuWarps / 4;
+  const int npieces = (nG + kGuPiece - 1) / kGuPiece;
+  const int ppw = npieces > wq ? (npieces - 1 - wq) / 4 + 1 : 0;   // pieces per item for this warp
+  const int q_items = my_items > quad ? (my_items - 1 - quad) / nquads + 1 : 0;
+  const int total = q_items * ppw;           // this warp's (item, piece) sequence
+  unsigned char* wst = smem + m.stages + (size_t)warp * spw * m.stage_bytes;
+  const size_t LO = kGuPiece * kTileRows * 8, HI = BITS == 3 ? kGuPiece * kTileRows * 4 : 0;
+  const size_t hwst = hw_expert_halves(Fmax, T);
+
+  auto issue = [&](int q) {   // sequence index q -> (item li, piece wq + 4*j); whole warp
+    const int li = q / ppw, p = wq + 4 * (q % ppw);
+    const int it = quad + li * nquads;
+    int u, tile;
+    gu_item(L, blockIdx.x + it * gridDim.x, Fs16, F16, &u, &tile);
+    gu_copy<BITS>(L, list, u, tile, p, wst + (size_t)(q % spw) * m.stage_bytes, ctl);
+  };
+  for (int q = 0; q < spw && q < total; ++q) issue(q);
+  int issued = spw < total ? spw : total;
+
+  int seq = 0;
+  for (int li = 0; li < q_items; ++li) {
+    float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < ppw; ++j, ++seq) {
+      const int s = seq % spw, p = wq + 4 * j;
+      cp_async_wait_upto(issued - 1 - seq);   // this piece's group has landed
+      __syncwarp();
+      {
+        const unsigned char* st = wst + (size_t)s * m.stage_bytes;
+        const __half* scg = reinterpret_cast<const __half*>(st + 2 * (LO + HI));
+        const __half* scu = scg + kGuPiece * kTileRows;
+        const int g0 = kGuPiece * p, np = min(kGuPiece, nG - g0);
+#pragma unroll 4
+        for (int c = 0; c < np; ++c) {
+          const uint4 xf = xs[(g0 + c) * 32 + lane];
+          const uint32_t b[4] = {xf.x, xf.y, xf.z, xf.w};
+          if (BITS == 2) {
+            const float2 cr = *reinterpret_cast<const float2*>(corr + (g0 + c) * kMaxDecodeT + 2 * (lane & 3));
+            group_mma_2b_offset(st, scg, c, b, cr, accg);
+            group_mma_2b_offset(st + LO + HI, scu, c, b, cr, accu);
+          } else {
+            group_mma<BITS>(st, st + LO, scg, c, b, accg);
+            group_mma<BITS>(st + LO + HI, st + 2 * LO + HI, scu, c, b, accu);
+          }
+        }
+      }
+      __syncwarp();
+      // the stage is free again: refill it with the piece spw steps ahead
+      if (issued < total) {
+        issue(issued);
+        ++issued;
+      }
+    }
+    float* pb = part + ((size_t)(quad * 2 + (li & 1)) * 4) * 32 * 8;
+    *reinterpret_cast<float4*>(pb + (wq * 32 + lane) * 8) = make_float4(accg[0], accg[1], accg[2], accg[3]);
+    *reinterpret_cast<float4*>(pb + (wq * 32 + lane) * 8 + 4) = make_float4(accu[0], accu[1], accu[2], accu[3]);
+    named_bar_sync(1 + quad, 128);
+    // warp wq finishes fragment element e = wq of every lane:
+    // row g + 8*(e>>1), token 2t + (e&1)
+    {
+      const int e = wq, g = lane >> 2, t = lane & 3;
+      const int n = 2 * t + (e & 1);
+      float gv = 0.f, up = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        gv += pb[(w * 32 + lane) * 8 + e];
+        up += pb[(w * 32 + lane) * 8 + 4 + e];
+      }
+      if (n < T) {
+        const int it = quad + li * nquads;
+        int u, tile;
+        gu_item(L, blockIdx.x + it * gridDim.x, Fs16, F16, &u, &tile);
+        const float hv = gv / (1.f + expf(-gv)) * up * list->w[u][n];
+        // the fp16 hidden value: out-of-range values are flagged (always on)
+        if (!(fabsf(hv) <= 65504.f)) record_error(ctl, kErrNonFinite, 0x402);
+        const int f = tile * kTileRows + g + 8 * (e >> 1);
+        const int c = f >> 5, kk = f & 31, mm = kk >> 3, tt = (kk & 7) >> 1, hh = kk & 1;
+        hw[(size_t)u * hwst + ((size_t)c * 4 * T + n * 4 + tt) * 8 + mm * 2 + hh] = __float2half_rn(hv);
+      }
+    }
+  }
+  cp_async_wait<0>();   // no copy may still be landing in this warp's stages
+}
+
+// ------------------------------------------------------------------- down
+struct DnSmem {
+  size_t bars, list, first, red, stages, total, stage_bytes, w_bytes;
+  int spw;
+};
+__host__ __device__ inline DnSmem dn_smem(int E, int bits, int Fmax, int T, int spw) {
+  DnSmem m;
+  size_t o = 0;
+  m.spw = spw;
+  m.bars = o;
+  o += (size_t)kDnWarps * spw * sizeof(uint64_t);
   o = (o + 15) & ~size_t(15);
   m.list = o;
   o += sizeof(ExpList);
@@ -284,574 +557,194 @@ __host__ __device__ inline DecSmem dec_smem(int d, int E, int bits, int nslots) 
   m.first = o;
   o += 2 * (size_t)E * sizeof(int);   // first-occurrence scratch, slot table
   o = (o + 15) & ~size_t(15);
-  m.sel = o;                                       // ids int32 [T][k], weights fp32 [T][k]
-  o += 2 * (size_t)kMaxDecodeT * 16 * 4;
+  m.red = o;
+  o += kDnWarps * 32 * 4 * sizeof(float);
   o = (o + 127) & ~size_t(127);
-  m.xs = o;                                        // B fragments of the tokens, per group
-  o += (size_t)nG * 32 * 16;
-  m.corr = o;                                      // 2-bit offset-form correction [group][token]
-  o += (size_t)nG * kMaxDecodeT * sizeof(float);   // (xs and corr: one bulk copy, in this order)
-  o = (o + 15) & ~size_t(15);
-  m.part = o;                                      // gate/up partial sums [warp][tile][lane][4]
-  o += (size_t)kDecWarps * 2 * 32 * 4 * sizeof(float);
-  m.hfrag = o;                                     // hidden slice as down B fragments [lane][4]
-  o += 32 * 4 * sizeof(uint32_t);
-  o = (o + 127) & ~size_t(127);
-  m.slots = o;
-  m.slot = ((size_t)dec_piece_bytes(d, bits) + 127) & ~size_t(127);
-  o += (size_t)nslots * m.slot;
+  m.stages = o;
+  const int nGF = Fmax / kGroup;
+  m.w_bytes = (size_t)nGF * kTileRows * group_bytes(bits) + (size_t)nGF * kTileRows * 2;
+  m.stage_bytes = m.w_bytes + hw_expert_halves(Fmax, T) * 2;
+  o += (size_t)kDnWarps * spw * m.stage_bytes;
   m.total = o;
   return m;
 }
 
-// Source of list position u (the shared expert when id < 0).
-struct ExpSrc {
-  const uint8_t* codes;
-  const uint16_t* scales;
-  int F;
-  int slot;   // TMA slot coordinate (0 for the shared expert)
-  bool shared;
-};
-__device__ __forceinline__ ExpSrc expert_src(const LayerDev& L, bool shared, int slot) {
-  ExpSrc r;
-  r.shared = shared;
-  if (shared) {
-    r.codes = L.scodes;
-    r.scales = L.sscales;
-    r.F = L.Fs;
-    r.slot = 0;
-  } else {
-    r.codes = L.codes + (long long)slot * L.cbe;
-    r.scales = L.scales + (long long)slot * L.nse;
-    r.F = L.F;
-    r.slot = slot;
-  }
-  return r;
-}
-
-// Request piece `kind` (0 = Wg slice, 1 = Wu slice, 2 = Wd group column) of
-// slice s of expert `src` into `dst`; completion on `bar` (one arrival plus the
-// piece's bytes).  One thread.
+// One CTA per 16-row tile of the output; warp w sums experts w, w+16, ...
+// through its private stages.  A stage holds expert u's Wd tile (requested as
+// soon as the routing is known, before this grid waits for the gate/up kernel)
+// and its hidden vector hw_u (requested after the wait): the stage barrier
+// expects two arrivals.  The warps' partial sums are added in a fixed order:
+// deterministic, no atomics.
 template <int BITS>
-__device__ __noinline__ void issue_piece(const DecMaps& maps, const LayerDev& L, const ExpSrc& src,
-                                            int s, int kind, unsigned char* dst, uint64_t* bar) {
-  const int d = L.d, nG = d / kGroup, gb = group_bytes(BITS);
-  mbar_arrive_expect_tx(bar, dec_piece_bytes(d, BITS));
-  if (kind < 2) {
-    const long long tcb = (long long)nG * kTileRows * gb;   // code bytes of a 16-row tile
-    const long long mcb = (long long)src.F * nG * gb;        // code bytes of an F x d matrix
-    const long long msc = (long long)src.F * nG;             // scales of an F x d matrix
-    bulk_g2s(dst, src.codes + kind * mcb + 2LL * s * tcb, (uint32_t)(2 * tcb), bar);
-    bulk_g2s(dst + 2 * tcb, src.scales + kind * msc + 2LL * s * kTileRows * nG,
-             (uint32_t)(2 * kTileRows * nG * 2), bar);
-  } else {
-    const CUtensorMap* lo = src.shared ? &maps.slo : &maps.lo;
-    const CUtensorMap* hi = src.shared ? &maps.shi : &maps.hi;
-    const CUtensorMap* sc = src.shared ? &maps.ssc : &maps.sc;
-    tma_load_4d(dst, lo, 0, s, 0, src.slot, bar);
-    if (BITS == 3) tma_load_4d(dst + 8 * d, hi, 0, s, 0, src.slot, bar);
-    tma_load_4d(dst + gb * d, sc, 0, s, 0, src.slot, bar);
-  }
-}
-
-// ------------------------------------------------------------ expert kernel
-// One CTA per SM (grid G).  Units in list order (the shared expert's slices
-// first, then each routed expert's in first-occurrence order of the window);
-// unit n runs on CTA n % G.  NRT: output-row tiles per warp (d / 256, rounded
-// up to 8 or 16).
-//
-// Warp roles inside a unit: gate/up -- warp w takes matrix w / 8 (Wg, Wu) and
-// the K-eighth w % 8 of both 16-row tiles of the slice, so each token fragment
-// it loads serves two tiles; the eight partial sums of a (matrix, tile) are
-// added in warp order.  Down -- warp w takes the output-row tiles w, w+16, ...
-// of the Wd group column and keeps their sums in registers across units.
-// The tokens' B fragments (and, for 2-bit, the offset-form corrections) come
-// precomputed from the router kernel: one bulk copy.
-// At most 88 registers per thread, so that a router or combine CTA can stay
-// resident beside it (programmatic dependent launch overlaps the kernels).
-template <int BITS, int NRT>
-__global__ void __maxnreg__(88)
-    decode_expert_kernel(const __grid_constant__ DecMaps maps, const __grid_constant__ LayerDev L,
-                         const unsigned char* __restrict__ xfrag, int T,
-                         const float* __restrict__ logits, const int32_t* __restrict__ ids_in,
-                         const float* __restrict__ w_in, int32_t* __restrict__ ids_out,
-                         float* __restrict__ w_out, float* __restrict__ partial, uint32_t flags,
-                         Control* ctl, int nslots) {
+__global__ void __launch_bounds__(kDnWarps * 32, 1)
+    decode_dn_kernel(LayerDev L, const uint16_t* __restrict__ x, int T,
+                     const int32_t* __restrict__ ids, const float* __restrict__ wts,
+                     const __half* __restrict__ hw, uint16_t* __restrict__ y, int Fmax,
+                     uint32_t flags, Control* ctl, int spw) {
   extern __shared__ __align__(128) unsigned char smem[];
-  const DecSmem m = dec_smem(L.d, L.E, BITS, nslots);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + m.bars);
+  const DnSmem m = dn_smem(L.E, BITS, Fmax, T, spw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + m.bars);
   ExpList* list = reinterpret_cast<ExpList*>(smem + m.list);
   int* first = reinterpret_cast<int*>(smem + m.first);
-  int* slot_s = first + L.E;
-  int32_t* sel_ids = reinterpret_cast<int32_t*>(smem + m.sel);
-  float* sel_w = reinterpret_cast<float*>(sel_ids + kMaxDecodeT * 16);
-  const uint4* xs = reinterpret_cast<const uint4*>(smem + m.xs);
-  const float* corr = reinterpret_cast<const float*>(smem + m.corr);
-  float* part = reinterpret_cast<float*>(smem + m.part);
-  __half* hfrag = reinterpret_cast<__half*>(smem + m.hfrag);
-  unsigned char* slots = smem + m.slots;
-  __shared__ __align__(8) uint64_t xbar;
-
+  float* red = reinterpret_cast<float*>(smem + m.red);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int d = L.d, nG = d / kGroup, gb = group_bytes(BITS);
-  const int G = gridDim.x;
-  const int sh_units = L.Fs / 32, Fu = L.F / 32;
-  const long long tcb = (long long)nG * kTileRows * gb;
-  auto slot_ptr = [&](int p) { return slots + (size_t)(p % nslots) * m.slot; };
-
+  const int d = L.d, tau = blockIdx.x;
   if (tid == 0) {
-    for (int s = 0; s < nslots; ++s) mbar_init(&full[s], 1);
-    mbar_init(&xbar, 1);
+    for (int s = 0; s < kDnWarps * spw; ++s) mbar_init(&bars[s], 2);
     fence_barrier_init();
   }
-  // the tensor-map descriptors in use into the TMA unit's cache
-  if (warp == 1 && lane < 6 && (BITS == 3 || lane % 3 != 1) && (lane < 3 || L.Fs > 0)) {
-    const CUtensorMap* mp = &maps.lo + lane;
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(mp)) : "memory");
-  }
-  expert_list_prologue(L, list, slot_s, first, ctl);
+  expert_list_prologue(L, list, first + L.E, first, ctl);
   __syncthreads();
+  // The routing lists were written two launches back (the router): readable
+  // before this grid waits on decode_gu.
+  if (warp == 0) build_expert_list(ids, wts, T, L, list, first + L.E, first, ctl);
+  __syncthreads();
+  const int n_exp = list->n;
+  const size_t hwst = hw_expert_halves(Fmax, T);
+  const int mine = n_exp > warp ? (n_exp - 1 - warp) / kDnWarps + 1 : 0;
+  unsigned char* wst = smem + m.stages + (size_t)warp * spw * m.stage_bytes;
+  uint64_t* wbar = bars + warp * spw;
 
-  // The shared expert's first unit does not depend on the routing: request it
-  // before waiting for the router.  Until the first unit's slices have landed
-  // only one unit is in flight, so that it is not queued behind the whole
-  // GPU's requests; then the ring fills up.
-  int issued = 0;   // pieces requested (thread 0)
-  int cap = 3;      // pieces allowed ahead of the consumer
-  if (tid == 0 && sh_units > (int)blockIdx.x) {
-    for (int p = 0; p < 3 && p < nslots; ++p) {
-      issue_piece<BITS>(maps, L, expert_src(L, true, 0), blockIdx.x, p, slot_ptr(p), &full[p]);
-      issued = p + 1;
-    }
-  }
-
-  pdl_wait();   // router logits (or the given routing) and the token fragments are complete
+  auto issue_w = [&](int j) {
+    const int u = warp + j * kDnWarps, s = j % spw;
+    const ExpSrc src = expert_src(L, list, u, ctl);
+    const int nGF = src.F / kGroup;
+    const size_t tcb = (size_t)nGF * kTileRows * group_bytes(BITS);
+    const size_t tsb = (size_t)nGF * kTileRows * 2;
+    const long long mcb = mat_codes_bytes(src.F, d, BITS);
+    unsigned char* st = wst + (size_t)s * m.stage_bytes;
+    mbar_arrive_expect_tx(&wbar[s], (uint32_t)(tcb + tsb));
+    bulk_g2s(st, src.codes + 2 * mcb + (long long)tau * tcb, (uint32_t)tcb, &wbar[s]);
+    bulk_g2s(st + tcb, src.scales + 2LL * src.F * (d / kGroup) + (long long)tau * kTileRows * nGF,
+             (uint32_t)tsb, &wbar[s]);
+  };
+  auto issue_h = [&](int j) {
+    const int u = warp + j * kDnWarps, s = j % spw;
+    const int F = list->id[u] < 0 ? L.Fs : L.F;
+    const uint32_t hb = (uint32_t)(F * T * 2);
+    mbar_arrive_expect_tx(&wbar[s], hb);
+    bulk_g2s(wst + (size_t)s * m.stage_bytes + m.w_bytes, hw + (size_t)u * hwst, hb, &wbar[s]);
+  };
+  const int pre = mine < spw ? mine : spw;
+  if (lane == 0)
+    for (int j = 0; j < pre; ++j) issue_w(j);
+  pdl_wait();   // hidden vectors come from decode_gu
   pdl_launch_dependents();
-  if (tid == 0) {
-    const uint32_t xb = (uint32_t)nG * (32 * 16 + kMaxDecodeT * 4);
-    mbar_arrive_expect_tx(&xbar, xb);
-    bulk_g2s(smem + m.xs, xfrag, xb, &xbar);
-  }
+  if (lane == 0)
+    for (int j = 0; j < pre; ++j) issue_h(j);
+  int issued = pre;
 
-  // ---- routing of the window (warps 0..T-1 select from the logits)
-  if (logits) {
-    if (warp < T) {
-      const float* row = logits + (size_t)warp * L.E;
-      if (L.E <= 512)
-        warp_topk_n<16>(row, L.E, L.k, sel_ids + warp * L.k, sel_w + warp * L.k, ctl, flags & MOE_F_DEBUG);
-      else
-        warp_topk_n<32>(row, L.E, L.k, sel_ids + warp * L.k, sel_w + warp * L.k, ctl, flags & MOE_F_DEBUG);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int j = 0; j < mine; ++j) {
+    const int u = warp + j * kDnWarps, s = j % spw;
+    if (!mbar_wait(&wbar[s], (j / spw) & 1, ctl, 0x501)) break;   // no barrier inside the loop
+    const int F = list->id[u] < 0 ? L.Fs : L.F;
+    const int nGF = F / kGroup;
+    const size_t tcb = (size_t)nGF * kTileRows * group_bytes(BITS);
+    const unsigned char* st = wst + (size_t)s * m.stage_bytes;
+    const __half* sc = reinterpret_cast<const __half*>(st + tcb);
+    const uint4* hws = reinterpret_cast<const uint4*>(st + m.w_bytes);
+#pragma unroll 4
+    for (int c = 0; c < nGF; ++c) {
+      uint4 bf = make_uint4(0, 0, 0, 0);
+      if (lane < 4 * T) bf = hws[c * 4 * T + lane];
+      const uint32_t b[4] = {bf.x, bf.y, bf.z, bf.w};
+      group_mma<BITS>(st, st + nGF * kTileRows * 8, sc, c, b, acc);
     }
-  } else {
-#pragma unroll 1
-    for (int i = tid; i < T * L.k; i += blockDim.x) {
-      sel_ids[i] = __ldcg(ids_in + i);
-      sel_w[i] = __ldcg(w_in + i);
-    }
-  }
-  __syncthreads();
-  if (warp == 0) build_expert_list(sel_ids, sel_w, T, L, list, slot_s, first, ctl);
-  __syncthreads();
-  if (blockIdx.x == 0 && ids_out) {
-    for (int i = tid; i < T * L.k; i += blockDim.x) {
-      ids_out[i] = sel_ids[i];
-      w_out[i] = sel_w[i];
-    }
-  }
-
-  const int n_units = sh_units + (list->n - (L.Fs > 0 ? 1 : 0)) * Fu;
-  if (blockIdx.x == 0 && tid == 0) ctl->decode_ctas = (uint32_t)(n_units < G ? n_units : G);
-  const int my = n_units > (int)blockIdx.x ? (n_units - 1 - (int)blockIdx.x) / G + 1 : 0;
-  const int npieces = 3 * my;
-  auto unit_src = [&](int j, int* s) {
-    const int n = blockIdx.x + j * G;
-    if (n < sh_units) {
-      *s = n;
-      return expert_src(L, true, 0);
-    }
-    const int u = (L.Fs > 0 ? 1 : 0) + (n - sh_units) / Fu;
-    *s = (n - sh_units) % Fu;
-    return expert_src(L, false, list->slot[u]);
-  };
-  auto unit_u = [&](int j) {
-    const int n = blockIdx.x + j * G;
-    return n < sh_units ? 0 : (L.Fs > 0 ? 1 : 0) + (n - sh_units) / Fu;
-  };
-  auto refill = [&](int consumed) {   // thread 0: keep the ring full, in consumption order
-    const int lim = consumed + (cap < nslots ? cap : nslots);
-    while (issued < npieces && issued < lim) {
-      int s;
-      const ExpSrc src = unit_src(issued / 3, &s);
-      issue_piece<BITS>(maps, L, src, s, issued % 3, slot_ptr(issued), &full[issued % nslots]);
+    __syncwarp();
+    if (issued < mine) {
+      if (lane == 0) {
+        fence_proxy_async_smem();
+        issue_w(issued);
+        issue_h(issued);
+      }
       ++issued;
     }
-  };
-  if (tid == 0) refill(0);
-  bool ok = mbar_wait(&xbar, 0, ctl, 0x600);
-
-  float accd[NRT][4];
-#pragma unroll
-  for (int i = 0; i < NRT; ++i) accd[i][0] = accd[i][1] = accd[i][2] = accd[i][3] = 0.f;
-  const int ntiles = d / kTileRows;
-  const int mat = warp >> 3, kq = warp & 7;
-  const int c0 = kq * nG / 8, c1 = (kq + 1) * nG / 8;
-  int j = 0;
-  for (; j < my; ++j) {
-    const int pg = 3 * j, pu = pg + 1, pd = pg + 2;
-    ok = ok && mbar_wait(&full[pg % nslots], (pg / nslots) & 1, ctl, 0x601);
-    ok = ok && mbar_wait(&full[pu % nslots], (pu / nslots) & 1, ctl, 0x602);
-    if (!__syncthreads_and(ok)) break;
-    if (j == 0 && tid == 0) {   // the first unit is here: let the ring fill
-      cap = nslots;
-      refill(0);
-    }
-    // gate/up: warp (matrix, K eighth), both tiles of the slice
-    {
-      const unsigned char* pc = slot_ptr(mat ? pu : pg);
-      const __half* sc = reinterpret_cast<const __half*>(pc + 2 * tcb);
-      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
-      for (int c = c0; c < c1; ++c) {
-        const uint4 xf = xs[c * 32 + lane];
-        const uint32_t b[4] = {xf.x, xf.y, xf.z, xf.w};
-        if (BITS == 2) {
-          const float2 cr = *reinterpret_cast<const float2*>(corr + c * kMaxDecodeT + 2 * (lane & 3));
-          group_mma_2b_offset(pc, sc, c, b, cr, a0);
-          group_mma_2b_offset(pc + tcb, sc + kTileRows * nG, c, b, cr, a1);
-        } else {
-          group_mma<BITS>(pc, pc + nG * kTileRows * 8, sc, c, b, a0);
-          group_mma<BITS>(pc + tcb, pc + tcb + nG * kTileRows * 8, sc + kTileRows * nG, c, b, a1);
-        }
-      }
-      float4* pw = reinterpret_cast<float4*>(part) + (warp * 2) * 32 + lane;
-      pw[0] = make_float4(a0[0], a0[1], a0[2], a0[3]);
-      pw[32] = make_float4(a1[0], a1[1], a1[2], a1[3]);
-    }
-    __syncthreads();
-    if (tid == 0) {   // the Wg and Wu slots are free
-      fence_proxy_async_smem();
-      refill(pg + 2);
-    }
-    // SwiGLU and routing weight: one (row, token) of the slice per thread
-    if (tid < 256) {
-      const int htl = tid >> 7, ln = (tid >> 2) & 31, e = tid & 3;
-      float gs = 0.f, us = 0.f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        gs += part[((q * 2 + htl) * 32 + ln) * 4 + e];
-        us += part[(((8 + q) * 2 + htl) * 32 + ln) * 4 + e];
-      }
-      const int row = (ln >> 2) + 8 * (e >> 1) + 16 * htl;   // hidden unit within the slice
-      const int n = 2 * (ln & 3) + (e & 1);                   // token
-      float h = 0.f;
-      if (n < T) h = gs / (1.f + expf(-gs)) * us * list->w[unit_u(j)][n];
-      if (!(fabsf(h) <= 65504.f)) record_error(ctl, kErrNonFinite, 0x603);
-      // down-projection B fragment: k = row, column = token; 2-bit offset
-      // form: the value divided by 4^(k / 8)
-      if (BITS == 2) h *= 1.f / (float)(1 << (2 * (row >> 3)));
-      const int tp = (row & 7) >> 1, jj = row >> 3, hh = row & 1;
-      hfrag[((n * 4 + tp) * 4 + jj) * 2 + hh] = __float2half_rn(h);
-    }
-    ok = mbar_wait(&full[pd % nslots], (pd / nslots) & 1, ctl, 0x604);
-    if (!__syncthreads_and(ok)) break;
-    // down: this warp's output-row tiles, one quantisation group each
-    {
-      const uint4 hb = reinterpret_cast<const uint4*>(hfrag)[lane];
-      const uint32_t b[4] = {hb.x, hb.y, hb.z, hb.w};
-      const unsigned char* pp = slot_ptr(pd);
-      const __half* dsc = reinterpret_cast<const __half*>(pp + gb * d);
-      if (BITS == 2) {
-        // offset-form correction of token g: sum over the group of
-        // B * (1024 + 2 * 4^m); this lane holds 8 of the 32 values (k = 2t +
-        // {0,1} + 8m), the four lanes t of the row group hold all of them
-        float cs = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const __half2 v = u32_as_h2(b[q]);
-          cs += (__low2float(v) + __high2float(v)) * (1024.f + 2.f * (float)(1 << (2 * q)));
-        }
-        cs += __shfl_xor_sync(0xffffffffu, cs, 1);
-        cs += __shfl_xor_sync(0xffffffffu, cs, 2);
-        const int t = lane & 3;
-        const float2 cr = make_float2(__shfl_sync(0xffffffffu, cs, 8 * t),
-                                      __shfl_sync(0xffffffffu, cs, 8 * t + 4));
-#pragma unroll
-        for (int i = 0; i < NRT; ++i) {
-          const int r = warp + kDecWarps * i;
-          if (r < ntiles) group_mma_2b_offset(pp + r * 128, dsc + r * kTileRows, 0, b, cr, accd[i]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < NRT; ++i) {
-          const int r = warp + kDecWarps * i;
-          if (r < ntiles)
-            group_mma<BITS>(pp + r * 128, pp + 8 * d + r * 64, dsc + r * kTileRows, 0, b, accd[i]);
-        }
-      }
-    }
-    __syncthreads();
-    if (tid == 0) {
-      fence_proxy_async_smem();
-      refill(pg + 3);   // the Wd slot is free
-    }
   }
-  if (tid == 0) {
-    // a wait ran out: let every requested copy land before the CTA exits
-    if (j < my)
-      for (int p = 3 * j; p < issued; ++p) mbar_wait(&full[p % nslots], (p / nslots) & 1, ctl, 0x605);
-    if (!ok) mbar_wait(&xbar, 0, ctl, 0x606);
-  }
-  // this CTA's partial sums: lane (g, t) of tile r holds rows g, g+8 and tokens 2t, 2t+1
-  if (my > 0) {
-    const int g = lane >> 2, t = lane & 3;
-    float* p0 = partial + ((size_t)blockIdx.x * T + 2 * t) * d + warp * kTileRows + g;
-    float* p1 = p0 + d;
-    const bool w0 = 2 * t < T, w1 = 2 * t + 1 < T;
-#pragma unroll
-    for (int i = 0; i < NRT; ++i) {
-      if (warp + kDecWarps * i >= ntiles) break;
-      const int o = i * kDecWarps * kTileRows;
-      if (w0) {
-        p0[o] = accd[i][0];
-        p0[o + 8] = accd[i][2];
-      }
-      if (w1) {
-        p1[o] = accd[i][1];
-        p1[o + 8] = accd[i][3];
-      }
-    }
-  }
-}
-
-// ----------------------------------------------------------- combine kernel
-// y[n][row] = sum over the expert CTAs c (ascending) of partial[c][n][row]
-// (+ x[n][row] with MOE_F_RESIDUAL), rounded once to bf16.  A CTA covers 8
-// output rows; its threads split the CTAs into CS strided subsets, and the
-// subsets' sums are added in subset order: a fixed order, independent of
-// scheduling.
-constexpr int kCombRows = 8;
-constexpr int kCombThreads = 256;
-__global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(
-    const float* __restrict__ partial, const uint16_t* __restrict__ x, uint16_t* __restrict__ y,
-    int T, int d, uint32_t flags, const Control* ctl) {
-  __shared__ float4 red[kCombThreads / 2 * 2];
-  // The next kernel of a window chain (the router of the next layer) reads
-  // nothing this grid or the expert grid writes before it waits itself.
-  pdl_launch_dependents();
-  pdl_wait();
-  const int nc = (int)*reinterpret_cast<const volatile uint32_t*>(&ctl->decode_ctas);
-  const int row0 = blockIdx.x * kCombRows;
-  const int CS = (kCombThreads / 2) / T;
-  const int tid = threadIdx.x, q = tid & 1, n = (tid >> 1) % T, cs = (tid >> 1) / T;
-  if (cs < CS) {
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float* p = partial + (size_t)n * d + row0 + 4 * q;
-    const size_t stride = (size_t)T * d;
-#pragma unroll 4
-    for (int c = cs; c < nc; c += CS) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(p + (size_t)c * stride));
-      a.x += v.x;
-      a.y += v.y;
-      a.z += v.z;
-      a.w += v.w;
-    }
-    red[(cs * T + n) * 2 + q] = a;
-  }
+  if (lane == 0)
+    for (int j = issued > spw ? issued - spw : 0; j < issued; ++j)
+      mbar_wait(&wbar[j % spw], (j / spw) & 1, ctl, 0x502);
+  *reinterpret_cast<float4*>(red + (warp * 32 + lane) * 4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
   __syncthreads();
-  if (tid < kCombRows * T) {
-    const int nn = tid / kCombRows, r = tid % kCombRows;
-    float v = 0.f;
-    for (int c = 0; c < CS; ++c) {
-      const float4 a = red[(c * T + nn) * 2 + (r >> 2)];
-      v += (r & 3) == 0 ? a.x : (r & 3) == 1 ? a.y : (r & 3) == 2 ? a.z : a.w;
+  if (tid < 128) {
+    const int r = tid >> 3, n = tid & 7;
+    if (n < T) {
+      const int l = (r & 7) * 4 + (n >> 1), idx = (r >> 3) * 2 + (n & 1);
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDnWarps; ++w) v += red[(w * 32 + l) * 4 + idx];
+      const int i = tau * kTileRows + r;
+      if (flags & MOE_F_RESIDUAL) v += bf16_bits_to_float(x[(size_t)n * d + i]);
+      __nv_bfloat16 bv = __float2bfloat16_rn(v);
+      y[(size_t)n * d + i] = *reinterpret_cast<uint16_t*>(&bv);
     }
-    const size_t i = (size_t)nn * d + row0 + r;
-    if (flags & MOE_F_RESIDUAL) v += bf16_bits_to_float(x[i]);
-    __nv_bfloat16 bv = __float2bfloat16_rn(v);
-    y[i] = *reinterpret_cast<uint16_t*>(&bv);
   }
 }
 
 // -------------------------------------------------------------- launcher
-// The stage ring takes what is left of 216 KB after the fixed regions (the
-// SM's 228 KB then still holds a combine or router CTA beside it, for the
-// programmatic overlap); at least two slots (a unit's Wg and Wu slices are
-// consumed together), at most eight.
-constexpr size_t kSmemPerBlockMax = 216 * 1024;
-constexpr int kMaxSlots = 8;
+constexpr size_t kGuSmemBudget = 215 * 1024;
+constexpr size_t kDnSmemBudget = 215 * 1024;
 
-static int dec_nslots(int d, int E, int bits) {
-  const DecSmem m0 = dec_smem(d, E, bits, 0);
-  if (m0.total >= kSmemPerBlockMax) return 0;
-  const size_t n = (kSmemPerBlockMax - m0.total) / m0.slot;
-  return n > (size_t)kMaxSlots ? kMaxSlots : (int)n;
-}
+// The stage counts above aim at the budgets; with one stage per warp a launch
+// may go up to the sm_100 opt-in maximum of shared memory per block (232448
+// bytes), less a margin for the kernels' static shared variables.
+constexpr size_t kSmemPerBlockMax = 232448 - 256;
 
+// Whether a T-token window of this layer fits the decode kernels: one stage per
+// warp must hold a whole expert's Wd tile and hidden vectors (16 warps), and
+// the gate/up kernel its token copies.  Wider experts take the prefill path.
 bool decode_fits(int d, int E, int Fmax, int bits, int T) {
-  (void)Fmax;
-  if (d <= 0 || E <= 0 || T < 1 || T > kMaxDecodeT || (bits != 2 && bits != 3)) return false;
-  return dec_nslots(d, E, bits) >= 2;
-}
-
-// ---- tensor maps of the Wd group columns, cached per layer
-static PFN_cuTensorMapEncodeTiled_v12000 dec_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    cudaGetLastError();
-  });
-  return fn;
-}
-
-// Wd of an expert with hidden size F in a codes array of `nslot` slots of
-// `cbe` bytes: lo plane [slot][tile][group][16 rows x 8 B], hi plane
-// [slot][tile][group][16 x 4 B] (3-bit), scales [slot][tile][group][16] fp16.
-// Box: group column s of all d/16 tiles of one slot.
-static bool dec_encode(CUtensorMap* lo, CUtensorMap* hi, CUtensorMap* sc, const uint8_t* codes,
-                       const uint16_t* scales, int d, int F, int bits, int nslot, long long cbe,
-                       long long nse) {
-  auto fn = dec_encode_fn();
-  if (!fn) return false;
-  const int gb = group_bytes(bits), nG = d / kGroup, nGF = F / kGroup, ntiles = d / kTileRows;
-  const long long mcb = (long long)F * nG * gb;   // code bytes of one F x d matrix
-  const cuuint64_t tile_b = (cuuint64_t)nGF * kTileRows * gb;
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  {
-    cuuint64_t dims[4] = {128, (cuuint64_t)nGF, (cuuint64_t)ntiles, (cuuint64_t)nslot};
-    cuuint64_t str[3] = {128, tile_b, (cuuint64_t)cbe};
-    cuuint32_t box[4] = {128, 1, (cuuint32_t)ntiles, 1};
-    if (fn(lo, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(codes + 2 * mcb), dims, str,
-           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return false;
-  }
-  if (bits == 3) {
-    cuuint64_t dims[4] = {64, (cuuint64_t)nGF, (cuuint64_t)ntiles, (cuuint64_t)nslot};
-    cuuint64_t str[3] = {64, tile_b, (cuuint64_t)cbe};
-    cuuint32_t box[4] = {64, 1, (cuuint32_t)ntiles, 1};
-    if (fn(hi, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
-           const_cast<uint8_t*>(codes + 2 * mcb + (long long)nGF * kTileRows * 8), dims, str, box,
-           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return false;
-  } else {
-    memset(hi, 0, sizeof(*hi));
-  }
-  {
-    cuuint64_t dims[4] = {16, (cuuint64_t)nGF, (cuuint64_t)ntiles, (cuuint64_t)nslot};
-    cuuint64_t str[3] = {32, (cuuint64_t)nGF * 32, (cuuint64_t)nse * 2};
-    cuuint32_t box[4] = {16, 1, (cuuint32_t)ntiles, 1};
-    if (fn(sc, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4,
-           const_cast<uint16_t*>(scales + 2LL * F * nG), dims, str, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return false;
-  }
-  return true;
-}
-
-// A small direct-mapped cache of encoded maps, keyed by the layer's pointers
-// and shape (encoding costs a few microseconds of host time per map).
-struct DecMapEntry {
-  const void *codes, *scales, *scodes, *sscales;
-  int d, E, F, Fs, bits;
-  DecMaps maps;
-};
-static std::mutex g_map_mu;
-static DecMapEntry g_map_cache[1024];
-
-static bool dec_maps(const LayerDev& L, DecMaps* out) {
-  const size_t h = ((reinterpret_cast<uintptr_t>(L.codes) >> 8) ^
-                    (reinterpret_cast<uintptr_t>(L.scales) >> 4) ^
-                    (reinterpret_cast<uintptr_t>(L.scodes) >> 6)) % 1024;
-  std::lock_guard<std::mutex> lock(g_map_mu);
-  DecMapEntry& e = g_map_cache[h];
-  if (e.codes == L.codes && e.scales == L.scales && e.scodes == L.scodes &&
-      e.sscales == L.sscales && e.d == L.d && e.E == L.E && e.F == L.F && e.Fs == L.Fs &&
-      e.bits == L.bits) {
-    *out = e.maps;
-    return true;
-  }
-  DecMaps mp;
-  memset(&mp, 0, sizeof(mp));
-  if (!dec_encode(&mp.lo, &mp.hi, &mp.sc, L.codes, L.scales, L.d, L.F, L.bits, L.E, L.cbe, L.nse))
+  if (d <= 0 || E <= 0 || Fmax <= 0 || T < 1 || T > kMaxDecodeT || (bits != 2 && bits != 3))
     return false;
-  if (L.Fs > 0) {
-    const long long cbs = 3LL * L.Fs * (L.d / kGroup) * group_bytes(L.bits);
-    const long long nss = 3LL * L.Fs * (L.d / kGroup);
-    if (!dec_encode(&mp.slo, &mp.shi, &mp.ssc, L.scodes, L.sscales, L.d, L.Fs, L.bits, 1, cbs, nss))
-      return false;
-  }
-  e.codes = L.codes;
-  e.scales = L.scales;
-  e.scodes = L.scodes;
-  e.sscales = L.sscales;
-  e.d = L.d;
-  e.E = L.E;
-  e.F = L.F;
-  e.Fs = L.Fs;
-  e.bits = L.bits;
-  e.maps = mp;
-  *out = mp;
-  return true;
+  return gu_smem(d, E, bits, 1).total <= kSmemPerBlockMax &&
+         dn_smem(E, bits, Fmax, T, 1).total <= kSmemPerBlockMax;
 }
 
-int decode_grid() {
-  const int g = sm_count();
-  return g < kMaxDecodeCtas ? g : kMaxDecodeCtas;
-}
-
-template <int BITS, int NRT>
-static cudaError_t launch_expert(const DecMaps& mp, const LayerDev& L, const unsigned char* xfrag, int T,
-                                 const float* logits, const int32_t* ids, const float* w,
-                                 int32_t* ids_out, float* w_out, float* partial, uint32_t flags,
-                                 Control* ctl, int nslots, cudaStream_t st) {
-  const DecSmem m = dec_smem(L.d, L.E, BITS, nslots);
-  cudaError_t e = cudaFuncSetAttribute(decode_expert_kernel<BITS, NRT>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)m.total);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(decode_expert_kernel<BITS, NRT>, dim3(decode_grid()), dim3(kDecWarps * 32),
-                    m.total, st, mp, L, xfrag, T, logits, ids, w, ids_out, w_out, partial, flags, ctl,
-                    nslots);
-}
-
-cudaError_t launch_decode(const LayerDev& L, const uint16_t* x, int T, const float* logits,
-                          const int32_t* ids, const float* w, int32_t* ids_out, float* w_out,
-                          uint16_t* y, uint32_t flags, char* ws, const WsLayout& lay,
-                          cudaStream_t st) {
+template <int BITS>
+static cudaError_t launch_decode_bits(const LayerDev& L, const uint16_t* x, int T,
+                                      const int32_t* ids, const float* w, uint16_t* y,
+                                      uint32_t flags, char* ws, const WsLayout& lay,
+                                      cudaStream_t st) {
   Control* ctl = reinterpret_cast<Control*>(ws + lay.ctl);
-  float* partial = reinterpret_cast<float*>(ws + lay.partial);
-  const unsigned char* xf = reinterpret_cast<const unsigned char*>(ws + lay.xfrag);
-  const int nslots = dec_nslots(L.d, L.E, L.bits);
-  if (nslots < 2) return cudaErrorInvalidValue;
-  DecMaps mp;
-  if (!dec_maps(L, &mp)) return cudaErrorInvalidValue;
-  cudaError_t e;
-  const bool wide = L.d / kTileRows > kDecWarps * 8;
-  if (L.bits == 2)
-    e = wide ? launch_expert<2, 16>(mp, L, xf, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st)
-             : launch_expert<2, 8>(mp, L, xf, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st);
-  else
-    e = wide ? launch_expert<3, 16>(mp, L, xf, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st)
-             : launch_expert<3, 8>(mp, L, xf, T, logits, ids, w, ids_out, w_out, partial, flags, ctl, nslots, st);
+  __half* hw = reinterpret_cast<__half*>(ws + lay.hw);
+  const int Fmax = L.F > L.Fs ? L.F : L.Fs;
+  const int max_exp = (T * L.k < L.E ? T * L.k : L.E) + (L.Fs > 0 ? 1 : 0);
+  // gate/up: private stages per warp, as many as fit (1..4)
+  int spw = 4;
+  GuSmem gm = gu_smem(L.d, L.E, BITS, spw);
+  while (gm.total > kGuSmemBudget && spw > 1) gm = gu_smem(L.d, L.E, BITS, --spw);
+  const int max_items = L.Fs / kTileRows + (max_exp - (L.Fs > 0 ? 1 : 0)) * (L.F / kTileRows);
+  int grid_gu = sm_count();
+  if (grid_gu > max_items) grid_gu = max_items;
+  cudaError_t e = cudaFuncSetAttribute(decode_gu_kernel<BITS>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gm.total);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_combine_kernel, dim3(L.d / kCombRows), dim3(kCombThreads), 0, st,
-                    static_cast<const float*>(partial), x, y, T, L.d, flags,
-                    static_cast<const Control*>(ctl));
+  e = launch_pdl(decode_gu_kernel<BITS>, dim3(grid_gu), dim3(kGuWarps * 32), gm.total, st, L, x, T,
+                 ids, w, hw, Fmax, flags, ctl, spw);
+  if (e != cudaSuccess) return e;
+  // down: enough private stages per warp to hold all its experts when they fit
+  int dspw = (max_exp + kDnWarps - 1) / kDnWarps;
+  if (dspw > 6) dspw = 6;
+  DnSmem dm = dn_smem(L.E, BITS, Fmax, T, dspw);
+  while (dm.total > kDnSmemBudget && dspw > 1) dm = dn_smem(L.E, BITS, Fmax, T, --dspw);
+  e = cudaFuncSetAttribute(decode_dn_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)dm.total);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(decode_dn_kernel<BITS>, dim3(L.d / kTileRows), dim3(kDnWarps * 32), dm.total,
+                    st, L, x, T, ids, w, static_cast<const __half*>(hw), y, Fmax, flags, ctl, dspw);
 }
 
-size_t decode_xfrag_bytes(const LayerDev& L) {
-  return (size_t)(L.d / kGroup) * (32 * 16 + kMaxDecodeT * 4);
+cudaError_t launch_decode(const LayerDev& L, const uint16_t* x, int T, const int32_t* ids,
+                          const float* w, uint16_t* y, uint32_t flags, char* ws, const WsLayout& lay,
+                          cudaStream_t st) {
+  if (L.bits == 2) return launch_decode_bits<2>(L, x, T, ids, w, y, flags, ws, lay, st);
+  return launch_decode_bits<3>(L, x, T, ids, w, y, flags, ws, lay, st);
 }
 
-size_t decode_partial_bytes(const LayerDev& L, int T) {
-  const int Tn = T < 1 ? 1 : (T > kMaxDecodeT ? kMaxDecodeT : T);
-  return (size_t)kMaxDecodeCtas * Tn * L.d * sizeof(float);
+size_t decode_hw_bytes(const LayerDev& L, int T) {
+  const int Fmax = L.F > L.Fs ? L.F : L.Fs;
+  const int max_exp = (T * L.k < L.E ? T * L.k : L.E) + (L.Fs > 0 ? 1 : 0);
+  return (size_t)max_exp * hw_expert_halves(Fmax, T) * sizeof(__half);
 }
 
 }  // namespace moe

@@ -35,8 +35,7 @@ struct WsLayout {
   size_t logits;     // fp32 [T][E]
   size_t ids;        // int32 [T][k]
   size_t w;          // fp32 [T][k]
-  size_t partial;    // decode: fp32 partial sums [expert CTAs][T][d]
-  size_t xfrag;      // decode: token operands of the expert kernel (B fragments, corrections)
+  size_t hw;         // decode: fp16 fragments [(U_max+1)][Fmax/32][32][8]
   size_t xn;         // prefill: bf16 [T][d] (PRENORM)
   size_t x16;        // prefill: fp16 [T][d]
   size_t counts;     // prefill: int32 [E+1]
@@ -54,31 +53,17 @@ struct WsLayout {
 WsLayout ws_layout(const LayerDev& L, int T);
 
 // launchers (return cudaError_t of the launch)
-// Router logits for a decode window (T <= 8): one warp per expert row; with
-// xfrag non-null it also writes the expert kernel's token operands there
-// (logits may be null: operands only).
-cudaError_t launch_router_gemv(const LayerDev& L, const uint16_t* x, int T, uint32_t flags,
-                               float* logits, unsigned char* xfrag, Control* ctl,
-                               cudaStream_t st);
-// Top-k selection and renormalised weights, one warp per token.
-cudaError_t launch_topk(const LayerDev& L, const float* logits, int T, int32_t* ids, float* w,
-                        uint32_t flags, Control* ctl, cudaStream_t st);
+cudaError_t launch_router_small(const LayerDev& L, const uint16_t* x, int T, uint32_t flags,
+                                float* logits, int32_t* ids, float* w, Control* ctl,
+                                cudaStream_t st);
 cudaError_t launch_router_large(const LayerDev& L, const uint16_t* x, int T, uint32_t flags,
                                 float* logits, int32_t* ids, float* w, uint16_t* wsplit,
                                 Control* ctl, cudaStream_t st);
 cudaError_t launch_router_tc(const LayerDev& L, const uint16_t* x, int T, float* logits,
                              uint16_t* hi, uint16_t* lo, Control* ctl, cudaStream_t st);
-// Expert CTAs of the decode step (one per SM, at most kMaxDecodeCtas); the
-// workspace holds one fp32 partial sum per CTA, token and output.
-constexpr int kMaxDecodeCtas = 160;
 bool decode_fits(int d, int E, int Fmax, int bits, int T);
-size_t decode_partial_bytes(const LayerDev& L, int T);
-size_t decode_xfrag_bytes(const LayerDev& L);
-// Decode expert step + combine.  Routing from `logits` (selected in the
-// kernel; ids_out / w_out receive it when non-null) or given (`ids`, `w`).
-cudaError_t launch_decode(const LayerDev& L, const uint16_t* x, int T, const float* logits,
-                          const int32_t* ids, const float* w, int32_t* ids_out, float* w_out,
-                          uint16_t* y, uint32_t flags, char* ws, const WsLayout& lay,
+cudaError_t launch_decode(const LayerDev& L, const uint16_t* x, int T, const int32_t* ids,
+                          const float* w, uint16_t* y, uint32_t flags, char* ws, const WsLayout& lay,
                           cudaStream_t st);
 cudaError_t launch_prefill(const LayerDev& L, const uint16_t* x, int T, const int32_t* ids,
                            const float* w, uint16_t* y, int32_t* offsets_out, int32_t* entries_out,

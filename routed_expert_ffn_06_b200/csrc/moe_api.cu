@@ -12,6 +12,7 @@ namespace moe {
 
 cudaError_t launch_prep_tokens(const uint16_t* x, int T, int d, uint32_t flags, uint16_t* xn,
                                __half* x16, Control* ctl, cudaStream_t st);
+size_t decode_hw_bytes(const LayerDev& L, int T);
 size_t prefill_ws_bytes(const LayerDev& L, int T, size_t* parts);
 
 namespace {
@@ -124,10 +125,8 @@ WsLayout ws_layout(const LayerDev& L, int T) {
   o += align256(Tn * L.k * sizeof(int32_t));
   w.w = o;
   o += align256(Tn * L.k * sizeof(float));
-  w.partial = o;
-  o += align256(decode_partial_bytes(L, T));
-  w.xfrag = o;
-  o += align256(decode_xfrag_bytes(L));
+  w.hw = o;
+  o += align256(decode_hw_bytes(L, T < kMaxDecodeT ? (int)Tn : kMaxDecodeT));
   w.decode_total = o;   // the decode path (router for T <= 8, decode step) uses no more
   if (T > 0) {
     size_t parts[16];
@@ -191,22 +190,10 @@ moe_status block_forward(const moe_layer* layer, const void* x_bf16, int32_t T, 
   }
   int32_t* ids = reinterpret_cast<int32_t*>(w + lay.ids);
   float* wt = reinterpret_cast<float*>(w + lay.w);
-  if (dec) {
-    // router logits, then the expert step selects from them (and records the
-    // routing in the workspace), then the combine
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    Control* ctl = reinterpret_cast<Control*>(w + lay.ctl);
-    float* logits = reinterpret_cast<float*>(w + lay.logits);
-    const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-    cudaError_t e = launch_router_gemv(L, x, T, flags, logits,
-                                       reinterpret_cast<unsigned char*>(w + lay.xfrag), ctl, st);
-    if (e == cudaSuccess)
-      e = launch_decode(L, x, T, logits, nullptr, nullptr, ids, wt, static_cast<uint16_t*>(y_bf16),
-                        flags, w, lay, st);
-    return from_cuda(e);
-  }
   s = moe_route_topk(layer, x_bf16, T, flags, nullptr, ids, wt, ws, ws_bytes, stream);
   if (s != MOE_OK) return s;
+  if (dec)
+    return moe_expert_ffn_decode(layer, x_bf16, T, ids, wt, y_bf16, flags, ws, ws_bytes, stream);
   return moe_expert_ffn_prefill(layer, x_bf16, T, ids, wt, y_bf16, nullptr, nullptr, flags, ws,
                                 ws_bytes, stream);
 }
@@ -261,11 +248,8 @@ moe_status moe_route_topk(const moe_layer* layer, const void* x_bf16, int32_t T,
   Control* ctl = reinterpret_cast<Control*>(w + lay.ctl);
   float* logits = logits_or_null ? logits_or_null : reinterpret_cast<float*>(w + lay.logits);
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-  if (T <= kMaxDecodeT) {
-    cudaError_t e = launch_router_gemv(L, x, T, flags, logits, nullptr, ctl, st);
-    if (e == cudaSuccess) e = launch_topk(L, logits, T, topk_ids, topk_w, flags, ctl, st);
-    return from_cuda(e);
-  }
+  if (T <= kMaxDecodeT)
+    return from_cuda(launch_router_small(L, x, T, flags, logits, topk_ids, topk_w, ctl, st));
   // large T: prenorm into xn first, the router reads bf16
   const uint16_t* xr = x;
   if (flags & MOE_F_PRENORM) {
@@ -295,17 +279,9 @@ moe_status moe_expert_ffn_decode(const moe_layer* layer, const void* x_bf16, int
   if (y_bf16 == x_bf16) return MOE_ERR_INVALID_ARG;
   if ((s = check_device()) != MOE_OK) return s;
   if (T == 0) return MOE_OK;
-  // the token operands of the expert kernel, then the expert step
-  char* w = static_cast<char*>(ws);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-  cudaError_t e = launch_router_gemv(L, x, T, flags, nullptr,
-                                     reinterpret_cast<unsigned char*>(w + lay.xfrag),
-                                     reinterpret_cast<Control*>(w + lay.ctl), st);
-  if (e == cudaSuccess)
-    e = launch_decode(L, x, T, nullptr, topk_ids, topk_w, nullptr, nullptr,
-                      static_cast<uint16_t*>(y_bf16), flags, w, lay, st);
-  return from_cuda(e);
+  return from_cuda(launch_decode(L, static_cast<const uint16_t*>(x_bf16), T, topk_ids, topk_w,
+                                 static_cast<uint16_t*>(y_bf16), flags, static_cast<char*>(ws), lay,
+                                 static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_expert_ffn_prefill(const moe_layer* layer, const void* x_bf16, int32_t T,

@@ -7,12 +7,11 @@
 // loop that must not call cudaMalloc (which synchronises the device) between
 // steps.  Every other entry point takes a caller-owned workspace.
 //
-// The scratch is one static array per device (kNoAllocScratchBytes, 8 MiB):
-// enough for the control block, logits, routing lists and the decode step's
-// per-CTA partial sums (160 x T x d fp32) of a T <= 4 window at the shapes of
-// the Strata layer (d = 2048, 512 experts, top-10: about 5.3 MB).  Larger
-// needs are rejected with MOE_ERR_WORKSPACE_TOO_SMALL before anything is
-// enqueued.
+// The scratch is one static array per device (kNoAllocScratchBytes, 2 MiB):
+// enough for the control block, logits, routing lists and decode partial sums
+// of a T <= 4 window at the shapes of the Strata layer (d = 2048, 512 experts,
+// ffn 512, top-10).  Larger needs are rejected with
+// MOE_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -21,7 +20,7 @@
 
 namespace moe {
 
-constexpr size_t kNoAllocScratchBytes = 8u << 20;
+constexpr size_t kNoAllocScratchBytes = 2u << 20;
 constexpr int kNoAllocMaxDevices = 64;
 
 // Zero at module load.  Each call also zeroes the control block at its start

@@ -22,7 +22,7 @@ constexpr float kRmsEps = 1e-6f;
 // instructions), and only the winning lane rescans.  NPER >= E / 32 logits per
 // lane.
 template <int NPER>
-__device__ __noinline__ void warp_topk_n(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
+__device__ void warp_topk_n(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
                             float* __restrict__ w, Control* ctl, bool debug) {
   const int lane = threadIdx.x & 31;
   // all loads first (independent, in flight together), checks afterwards

@@ -114,30 +114,29 @@ def test_status_strings(lib):
     assert "sm_100a" in moe.moe_build_info()
 
 
-def test_decode_takes_every_valid_width(lib):
-    """The decode step streams each expert in 32-row slices, so the width of
-    the experts does not bound it: the widest experts (ffn 4096) and the widest,
-    largest layer (d 4096, 1024 experts, 3-bit, top-16, an 8-token window) pass
-    every host check and stop at the missing device."""
+def test_decode_rejects_experts_too_wide_for_its_stages(lib):
+    """The decode step checks that its shared-memory stages hold the layer
+    before anything else touches the device: ffn 4096 at d 256 is a valid layer
+    that only the prefill step takes (MOE_ERR_UNSUPPORTED_SHAPE, not a launch
+    failure), while ffn 512 passes the shape checks and stops at the missing
+    device."""
     x, y, ids, w, ws = 0x7F0000400000, 0x7F0000500000, 0x7F0000700000, 0x7F0000800000, 0x7F0000600000
     wide = _layer(d_model=256, n_experts=20, ffn=4096, shared_ffn=4096, top_k=16)
-    assert lib.moe_expert_ffn_decode(ctypes.byref(wide), x, 1, ids, w, y, 0, ws, 1 << 30, None) == 8
-    big = _layer(d_model=4096, n_experts=1024, ffn=4096, shared_ffn=4096, top_k=16, bits=3)
-    assert lib.moe_expert_ffn_decode(ctypes.byref(big), x, 8, ids, w, y, 0, ws, 1 << 30, None) == 8
-    assert lib.moe_expert_ffn_decode(ctypes.byref(big), x, 9, ids, w, y, 0, ws, 1 << 30, None) == 2
+    assert lib.moe_expert_ffn_decode(ctypes.byref(wide), x, 1, ids, w, y, 0, ws, 1 << 30, None) == 2
+    ok = _layer(d_model=256, n_experts=20, ffn=512, shared_ffn=512, top_k=16)
+    assert lib.moe_expert_ffn_decode(ctypes.byref(ok), x, 8, ids, w, y, 0, ws, 1 << 30, None) == 8
 
 
-def test_block_forward_path_choice_by_window(lib):
-    """Path choice on the host, seen through the workspace it demands: windows
-    of up to 8 tokens run the decode path, which needs only a leading part of
-    the workspace (one byte short of the full size passes and the call stops at
-    the missing device, status 8); 9 tokens take the prefill path, which needs
-    it all (status 3)."""
+def test_block_forward_takes_prefill_for_experts_too_wide_for_decode(lib):
+    """Path choice on the host, seen through the workspace it demands: a
+    4-token window of a layer within the decode kernels' width runs the decode
+    path, which needs only a leading part of the workspace (so one byte short
+    of the full size passes and the call stops at the missing device); with
+    ffn 4096 the same window takes the prefill path, which needs it all."""
     x, y = 0x7F0000400000, 0x7F0000500000
-    for ffn in (512, 4096):
+    for ffn, want in [(512, 8), (4096, 3)]:
         L = _layer(d_model=256, n_experts=20, ffn=ffn, shared_ffn=ffn, top_k=16)
-        for T, want in [(4, 8), (8, 8), (9, 3)]:
-            full = lib.moe_workspace_bytes(ctypes.byref(L), T)
-            assert full > 0
-            rc = lib.moe_block_forward(ctypes.byref(L), x, T, y, 0, 0x7F0000600000, full - 1, None)
-            assert rc == want, (ffn, T, rc)
+        full = lib.moe_workspace_bytes(ctypes.byref(L), 4)
+        assert full > 0
+        rc = lib.moe_block_forward(ctypes.byref(L), x, 4, y, 0, 0x7F0000600000, full - 1, None)
+        assert rc == want, (ffn, rc)

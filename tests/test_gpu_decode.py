@@ -168,9 +168,9 @@ def test_decode_wide_model(T):
 
 @pytest.mark.parametrize("T,F", [(1, 1920), (8, 640)])
 def test_decode_widest_experts_it_takes(T, F):
-    """Wide experts (routed and shared, ffn 1920 and 640) for a 1- and an
-    8-token window, with the largest top-k (16): routing and outputs match the
-    oracle."""
+    """The widest experts (routed and shared) the decode kernels take for a 1-
+    and an 8-token window, with the largest top-k (16): routing and outputs
+    match the oracle."""
     sh = synth.MoEShape(d=256, E=20, F=F, Fs=F, k=16, bits=2)
     layer = synth.make_layer(sh, seed=15, device="cuda", bias="normal")
     x = synth.make_tokens(T, sh.d, seed=16 + T, device="cuda")
@@ -182,18 +182,20 @@ def test_decode_widest_experts_it_takes(T, F):
 
 
 @pytest.mark.parametrize("T", [1, 8])
-def test_widest_experts_take_the_decode_step(T):
-    """The widest experts the shape checks accept (ffn 4096, routed and shared,
-    top-16): the decode step streams them in 32-row slices, matches the oracle,
-    and the block forward gives the same bytes."""
+def test_wide_experts_take_the_prefill_step(T):
+    """Experts too wide for the decode kernels' stages (ffn 4096): the decode
+    call rejects the shape before enqueuing anything, and the block forward
+    runs the prefill step instead, matching the oracle."""
     sh = synth.MoEShape(d=256, E=20, F=4096, Fs=4096, k=16, bits=2)
     layer = synth.make_layer(sh, seed=15, device="cuda", bias="normal")
     x = synth.make_tokens(T, sh.d, seed=16 + T, device="cuda")
     gb = GpuBlock(layer, T)
     logits, ids, w = gb.route(x)
-    y = gb.decode(x, ids, w)
+    with pytest.raises(moe.MoEError) as err:
+        gb.decode(x, ids, w)
+    assert err.value.status == 2          # MOE_ERR_UNSUPPORTED_SHAPE
+    y = gb.block(x)
     oracle_check(layer, x, logits, ids, w, y)
-    assert torch.equal(gb.block(x), y)
     assert gb.error_word() == (0, 0)
 
 

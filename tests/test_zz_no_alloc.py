@@ -4,7 +4,7 @@ with no device allocator, a step loop that must not call cudaMalloc because it
 synchronises the device).  Called through the C ABI, it must give exactly the
 bytes of the workspace entry point (moe_block_forward: same kernels, same
 inputs), on calls in a row and on calls queued back to back on one stream with
-no host synchronisation between them, and reject what its 8 MiB scratch cannot
+no host synchronisation between them, and reject what its 2 MiB scratch cannot
 hold before enqueuing anything.
 
 This file sorts last so that a run stopping at its first failure has already
@@ -101,10 +101,10 @@ def test_noalloc_rejects_long_windows_and_large_shapes():
     x = synth.make_tokens(8, 64, seed=1, device="cuda")
     y = torch.empty_like(x)
     assert _status(L, x, 5, y) == 2            # MOE_ERR_UNSUPPORTED_SHAPE: T > 4
-    # a layer whose decode workspace exceeds 8 MiB (d 4096, 1024 experts, ffn 4096,
+    # a layer whose decode workspace exceeds 2 MiB (d 4096, 1024 experts, ffn 4096,
     # top-16, 3-bit): rejected by size before any weight is read
     big = moe.moe_layer(4096, 1024, 4096, 16, 3, 32, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 4096)
-    assert moe.moe_workspace_bytes(big, 4) > (8 << 20)
+    assert moe.moe_workspace_bytes(big, 4) > (2 << 20)
     xb = torch.zeros(4, 4096, dtype=torch.bfloat16, device="cuda")
     yb = torch.empty_like(xb)
     assert _status(big, xb, 4, yb) == 3        # MOE_ERR_WORKSPACE_TOO_SMALL
