@@ -45,10 +45,12 @@ def parse():
     p.add_argument("--workload", default="decode", choices=["decode", "prefill", "stack", "mix"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--layers", type=int, default=32, help="independent layer copies rotated")
+    p.add_argument("--rounds", type=int, default=2048,
+                   help="rounds of the T=1..4 windows in one decode step (smaller for profiling)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-prefill", action="store_true",
                    help="decode workload only (no prefill object in the line)")
-    p.add_argument("--prefill-steps", type=int, default=20)
+    p.add_argument("--prefill-steps", type=int, default=500)
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     return p.parse_args()
 
@@ -192,7 +194,6 @@ def measured_traffic(name: str):
 
 # ------------------------------------------------------------------ decode
 DECODE_WINDOWS = (1, 2, 3, 4)
-DECODE_ROUNDS = 2048        # rounds of the four windows in one step of the decode bench
 PREFILL_LAUNCHES = 11       # split router, router GEMM, top-k, prep, hist, scan, scatter,
                             # gather, GEMM1, GEMM2, combine per 8192-token chunk
 WORKLOAD_DECODE = ("decode single layer: d=2048, 512 experts ffn=512 + shared ffn=512, top-10, "
@@ -239,7 +240,7 @@ def bench_decode(args, rank, world, local):
     NL = args.layers
     K = args.steps if args.steps is not None else 20
     W = args.warmup if args.warmup is not None else 5
-    R = DECODE_ROUNDS                      # rounds of the four windows per step
+    R = args.rounds                        # rounds of the four windows per step
     nwin = len(DECODE_WINDOWS)
     ntok_step = R * sum(DECODE_WINDOWS)
     t_gen = time.time()
