@@ -45,6 +45,16 @@ def parse():
     p.add_argument("--workload", default="decode", choices=["decode", "prefill", "stack", "mix"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--layers", type=int, default=32, help="independent layer copies rotated")
+    p.add_argument("--topk", type=int, default=None,
+                   help="decode: experts per token (the pages' 'Faster' mode is top_k - 1)")
+    p.add_argument("--prefer-hot", type=int, default=0,
+                   help="decode: a selection bonus on each layer's N most popular experts")
+    p.add_argument("--prefer-bonus", type=float, default=0.5)
+    p.add_argument("--adapt-every", type=int, default=0,
+                   help="mix: re-order every layer's slots by its decayed routing counts every N "
+                        "decode steps (0: frozen layout)")
+    p.add_argument("--adapt-swaps", type=int, default=96)
+    p.add_argument("--adapt-decay", type=float, default=0.5)
     p.add_argument("--rounds", type=int, default=2048,
                    help="rounds of the T=1..4 windows in one decode step (smaller for profiling)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -237,6 +247,9 @@ def bench_decode(args, rank, world, local):
     moe.load()
     wl = synth.WORKLOADS["decode"]
     sh = wl["shape"]
+    if args.topk:
+        import dataclasses
+        sh = dataclasses.replace(sh, k=args.topk)
     NL = args.layers
     K = args.steps if args.steps is not None else 20
     W = args.warmup if args.warmup is not None else 5
@@ -247,7 +260,11 @@ def bench_decode(args, rank, world, local):
     layers = [synth.make_layer(sh, seed=rank * 1000 + i, layer=i, device=dev, bias=wl["bias"],
                                slot=wl["slot"]) for i in range(NL)]
     t_gen = time.time() - t_gen
-    structs = [moe.make_layer_struct(l) for l in layers]
+    prefs = [None] * NL
+    if args.prefer_hot:   # selection bonus on each layer's hottest experts (rank 1..N)
+        prefs = [torch.where(l.rank.to(dev) <= args.prefer_hot, args.prefer_bonus, 0.0).float()
+                 for l in layers]
+    structs = [moe.make_layer_struct(l, p) for l, p in zip(layers, prefs)]
     ws = moe.alloc_workspace(structs[0], max(DECODE_WINDOWS))
     # fresh tokens for every window of a step
     xs = [[synth.make_tokens(T, sh.d, seed=rank * 1000 + 7, step=r * nwin + i, device=dev)
@@ -400,6 +417,8 @@ def bench_decode(args, rank, world, local):
                    "parallelism": f"replicas x{world}",
                    "mma": "f16 x f16 -> f32 (weights dequantised in registers)",
                    "unique_experts_per_window": U_mean, "zipf_s_fitted": round(zipf_s, 3),
+                   "top_k": sh.k, "prefer_hot": args.prefer_hot,
+                   "prefer_bonus": args.prefer_bonus if args.prefer_hot else None,
                    "weights_gen_s": round(t_gen, 1)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -737,8 +756,14 @@ def bench_mix(args, rank, world, local):
     t_gen = time.time()
     layers = _stack_layers(wl, rank, dev)
     t_gen = time.time() - t_gen
-    structs = [moe.make_layer_struct(l) for l in layers]
+    AE = args.adapt_every
+    counts = [torch.zeros(sh.E, dtype=torch.float32, device=dev) if AE else None for _ in layers]
+    structs = [moe.make_layer_struct(l, route_counts=c) for l, c in zip(layers, counts)]
     ws = moe.alloc_workspace(structs[0], C)
+    if AE:
+        n = moe.moe_adapt_workspace_bytes(structs[0], args.adapt_swaps)
+        aws = torch.zeros(n + 256, dtype=torch.uint8, device=dev)
+        aws = aws[(-aws.data_ptr()) % 256:]
     flags = moe.F_PRENORM | moe.F_RESIDUAL
     stream = torch.cuda.Stream(device=dev)
     biases = [[l.router_bias.clone()] + [synth.permute_profile(l, seed=rank * 1000, epoch=e + 1)
@@ -782,6 +807,10 @@ def bench_mix(args, rank, world, local):
             for s in range(DS):
                 if s % drift == 0:
                     set_epoch(s // drift)
+                if AE and s > 0 and s % AE == 0:
+                    for L in structs:
+                        moe.moe_adapt_layout(L, args.adapt_decay, args.adapt_swaps, None, aws,
+                                             stream)
                 graphs[s % G].replay()
             d1.record(stream)
         stream.synchronize()
@@ -806,6 +835,8 @@ def bench_mix(args, rank, world, local):
                    "tokens": ntok, "weights_gb": round(NLy * (sh.E * eb + eb + sh.E * sh.d * 4) / 1e9, 2),
                    "l2": "inputs larger than L2 (34 GB of weights)",
                    "weights_gen_s": round(t_gen, 1), "parallelism": f"replicas x{world}"},
+        "adaptive_layout": ({"every_steps": AE, "max_swaps": args.adapt_swaps,
+                             "decay": args.adapt_decay} if AE else None),
         "prefill_tokens_per_s": round(NC * C * world / (ms_pf / 1e3), 1),
         "decode_tokens_per_s": round(DS * T * world / (ms_dec / 1e3), 1),
         "roofline": {"bound": "tensor", "achieved": round(flops / (ms_pf / 1e3) / 1e12, 1),

@@ -14,8 +14,9 @@
  *
  * Per token x (bf16, d values):
  *   logits[e] = sum_i x[i] * Wr[e][i] + b[e]                       (fp32)
- *   ids       = the top_k largest logits, largest first, equal logits ->
- *               lower expert index, NaN below every number
+ *   ids       = the top_k largest logits (plus router_pref, when given),
+ *               largest first, equal values -> lower expert index, NaN below
+ *               every number
  *   w[j]      = exp(logits[ids[j]] - logits[ids[0]]) / sum over the selected
  *   FFN_e(x)  = Wd_e (silu(Wg_e x) * (Wu_e x)),  silu(z) = z / (1 + e^-z)
  *   y         = FFN_shared(x) + sum_j w[j] * FFN_{ids[j]}(x)   -> bf16
@@ -110,6 +111,21 @@ typedef struct {
   const uint16_t* scales;       /* dev fp16 bits [E slots][3*F*d/32] */
   const uint8_t* shared_codes;  /* dev [3*Fs*d/32*(8|12)] or NULL when Fs == 0 */
   const uint16_t* shared_scales;/* dev fp16 bits [3*Fs*d/32] or NULL when Fs == 0 */
+  /* dev fp32 [E] or NULL: a per-expert selection bonus.  The selection ranks
+   * logits[e] + router_pref[e] (fp32 add; same tie and NaN rules), while the
+   * weights stay the softmax of the selected experts' logits.  This is the
+   * pages' "the router prefers experts already on the card" (release 0.2.7 in
+   * "Strata: a 12GB card runs 125B -- how the three storage tiers are
+   * squeezed out", section 4, "how to choose against Ollama / LM Studio /
+   * llama.cpp"): a positive bonus on a preferred set of experts.  NULL =
+   * plain top-k. */
+  const float* router_pref;
+  /* dev fp32 [E] or NULL: routing counters for the adaptive slot layout.
+   * When given, every selection made by the router (moe_route_topk and the
+   * block forward) adds 1.0 to route_counts[expert] (atomic adds of ones:
+   * exact below 2^24); moe_adapt_layout reads and decays them.  Selections
+   * passed in by the caller (the expert-step calls) are not counted. */
+  float* route_counts;
 } moe_layer;
 
 /* Bytes of workspace the calls below need for up to max_tokens tokens
@@ -198,6 +214,29 @@ moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t
  *    current sm_100 device). */
 moe_status moe_block_forward_noalloc(const moe_layer* layer, const void* x_bf16, int32_t T,
                                      void* y_bf16, uint32_t flags, void* stream);
+
+/* Adaptive frequency-ordered slot layout.  The pages' expert cache keeps
+ * counting the routing with exponential decay and swaps new hot experts in, at
+ * most 96 swaps per 4 rounds ("Strata: Run a 125B Model on a 12 GB GPU with
+ * MoE Expert Hot Cache", section "How It Works"; "Strata illustrated",
+ * section on the expert cache).  With every expert in HBM the "cache" is the
+ * slot order: this call ranks the experts by layer->route_counts (descending,
+ * equal counts by lower expert index), walks the ranks and swaps the expert
+ * of rank r into slot r until max_swaps swaps are made, moves the packed
+ * bytes (codes and scales) of the affected slots, rewrites expert_slot, and
+ * multiplies every count by decay (0 <= decay <= 1).  Results of the block do
+ * not depend on the slot order, so outputs stay bit-identical.
+ *  - Rewrites layer->codes, ->scales and ->expert_slot in place (they must be
+ *    writable device memory) and layer->route_counts (required).
+ *  - ws: at least moe_adapt_workspace_bytes(layer, max_swaps) bytes,
+ *    256-byte aligned (staging for 2*max_swaps slots).
+ *  - swaps_done_or_null: dev int32, receives the number of swaps made.
+ *  - Enqueued on stream after the work before it, without programmatic
+ *    overlap; a slot table that is not a permutation moves nothing and sets
+ *    the range bit in the workspace's error word (moe_workspace_error). */
+size_t moe_adapt_workspace_bytes(const moe_layer* layer, int32_t max_swaps);
+moe_status moe_adapt_layout(const moe_layer* layer, float decay, int32_t max_swaps,
+                            int32_t* swaps_done_or_null, void* ws, size_t ws_bytes, void* stream);
 
 const char* moe_status_string(moe_status status);
 

@@ -19,6 +19,8 @@ struct LayerDev {
   const uint16_t* scales;
   const uint8_t* scodes;
   const uint16_t* sscales;
+  const float* pref;   // selection bonus [E] or nullptr
+  float* counts;       // routing counters [E] or nullptr
   long long cbe;   // codes bytes per routed expert
   long long nse;   // scales per routed expert
 };

@@ -81,6 +81,8 @@ LayerDev to_dev(const moe_layer* l) {
   L.scales = l->scales;
   L.scodes = l->shared_codes;
   L.sscales = l->shared_scales;
+  L.pref = l->router_pref;
+  L.counts = l->route_counts;
   L.cbe = 3LL * L.F * L.d / kGroup * group_bytes(L.bits);
   L.nse = 3LL * L.F * L.d / kGroup;
   return L;

@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_small_kernel(
   __syncthreads();
   if (!s_last) return;
   for (int t = warp; t < T; t += kRouterWarps)
-    warp_topk(logits + (size_t)t * L.E, L.E, L.k, ids + (size_t)t * L.k, wout + (size_t)t * L.k,
+    warp_topk(logits + (size_t)t * L.E, L.pref, L.counts, L.E, L.k, ids + (size_t)t * L.k, wout + (size_t)t * L.k,
               ctl, flags & MOE_F_DEBUG);
   if (threadIdx.x == 0) atomicExch(&ctl->router_done, 0u);
 }
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerDev L, const float* __re
   pdl_launch_dependents();
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
-  warp_topk(logits + (size_t)t * L.E, L.E, L.k, ids + (size_t)t * L.k, w + (size_t)t * L.k, ctl,
+  warp_topk(logits + (size_t)t * L.E, L.pref, L.counts, L.E, L.k, ids + (size_t)t * L.k, w + (size_t)t * L.k, ctl,
             flags & MOE_F_DEBUG);
 }
 

@@ -21,23 +21,28 @@ constexpr float kRmsEps = 1e-6f;
 // the warp maximum of the keys and the lowest index holding it (two redux
 // instructions), and only the winning lane rescans.  NPER >= E / 32 logits per
 // lane.
-template <int NPER>
-__device__ void warp_topk_n(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
+template <int NPER, bool PREF>
+__device__ void warp_topk_n(const float* __restrict__ row, const float* __restrict__ pref,
+                            float* __restrict__ counts, int E, int k, int32_t* __restrict__ ids,
                             float* __restrict__ w, Control* ctl, bool debug) {
   const int lane = threadIdx.x & 31;
   // all loads first (independent, in flight together), checks afterwards
-  float v[NPER];
+  float v[NPER], b[PREF ? NPER : 1];
 #pragma unroll
   for (int i = 0; i < NPER; ++i) {
     const int e = lane + 32 * i;
     v[i] = e < E ? __ldcg(row + e) : 0.f;
+    if (PREF) b[i] = e < E ? __ldg(pref + e) : 0.f;
   }
+  // selection key: the logit, plus the expert's selection bonus when given
+  // (fp32 add); the weights below use the logits alone
   uint32_t key[NPER];
   bool bad = false;
 #pragma unroll
   for (int i = 0; i < NPER; ++i) {
-    key[i] = order_key(v[i]);
-    bad |= (lane + 32 * i < E) && !isfinite(v[i]);
+    const int e = lane + 32 * i;
+    key[i] = order_key(PREF ? v[i] + b[PREF ? i : 0] : v[i]);
+    bad |= (e < E) && !isfinite(v[i]);
   }
   if (debug && bad) record_error(ctl, kErrNonFinite, 0x100);
   uint32_t taken = 0;
@@ -67,32 +72,74 @@ __device__ void warp_topk_n(const float* __restrict__ row, int E, int k, int32_t
   };
   rescan();
   float my_v = 0.f;
+  uint32_t my_id = 0;
   for (int j = 0; j < k; ++j) {
     const uint32_t mk = __reduce_max_sync(0xffffffffu, bi == 0xFFFFFFFFu ? 0u : bk);
     const uint32_t win = __reduce_min_sync(0xffffffffu, (bi != 0xFFFFFFFFu && bk == mk) ? bi : 0xFFFFFFFFu);
     const uint32_t u = (mk & 0x80000000u) ? (mk & 0x7FFFFFFFu) : ~mk;
-    if (lane == j) my_v = __uint_as_float(u);
+    if (PREF) {   // the unbiased logit of the pick, from the lane that holds it
+      float own = 0.f;
+#pragma unroll
+      for (int i = 0; i < NPER; ++i)
+        if ((win >> 5) == (uint32_t)i) own = v[i];
+      const float vj = __shfl_sync(0xffffffffu, own, win & 31u);
+      if (lane == j) my_v = vj;
+    } else if (lane == j) {
+      my_v = __uint_as_float(u);
+    }
+    if (lane == j) my_id = win;
     if (lane == 0) ids[j] = static_cast<int32_t>(win);
     if ((win & 31u) == (uint32_t)lane) {
       taken |= 1u << (win >> 5);
       rescan();
     }
   }
-  const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
+  // softmax reference: the largest selected logit (the first pick without a
+  // selection bonus; with one, the picks are re-read unbiased and maximised)
+  float v0;
+  if (PREF) {
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, lane < k ? order_key(my_v) : 0u);
+    v0 = __uint_as_float((mk & 0x80000000u) ? (mk & 0x7FFFFFFFu) : ~mk);
+  } else {
+    v0 = __shfl_sync(0xffffffffu, my_v, 0);
+  }
+  // routing counters (adaptive slot layout): one count per pick
+  if (counts && lane < k) atomicAdd(counts + my_id, 1.f);
   const float ex = lane < k ? expf(my_v - v0) : 0.f;
   const float den = warp_sum(ex);
   if (lane < k) w[lane] = ex / den;
 }
 
-__device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, int k,
+// The variants with a selection bonus are kept out of line: their extra
+// register arrays then leave the plain path's allocation alone.
+template <int NPER>
+__device__ __noinline__ void warp_topk_pref(const float* __restrict__ row,
+                                            const float* __restrict__ pref,
+                                            float* __restrict__ counts, int E, int k,
+                                            int32_t* __restrict__ ids, float* __restrict__ w,
+                                            Control* ctl, bool debug) {
+  warp_topk_n<NPER, true>(row, pref, counts, E, k, ids, w, ctl, debug);
+}
+
+__device__ __forceinline__ void warp_topk(const float* __restrict__ row, const float* __restrict__ pref,
+                                          float* __restrict__ counts, int E, int k,
                                           int32_t* __restrict__ ids, float* __restrict__ w,
                                           Control* ctl, bool debug) {
-  if (E <= 128)
-    warp_topk_n<4>(row, E, k, ids, w, ctl, debug);
-  else if (E <= 512)
-    warp_topk_n<16>(row, E, k, ids, w, ctl, debug);
-  else
-    warp_topk_n<32>(row, E, k, ids, w, ctl, debug);
+  if (pref) {
+    if (E <= 128)
+      warp_topk_pref<4>(row, pref, counts, E, k, ids, w, ctl, debug);
+    else if (E <= 512)
+      warp_topk_pref<16>(row, pref, counts, E, k, ids, w, ctl, debug);
+    else
+      warp_topk_pref<32>(row, pref, counts, E, k, ids, w, ctl, debug);
+  } else {
+    if (E <= 128)
+      warp_topk_n<4, false>(row, pref, counts, E, k, ids, w, ctl, debug);
+    else if (E <= 512)
+      warp_topk_n<16, false>(row, pref, counts, E, k, ids, w, ctl, debug);
+    else
+      warp_topk_n<32, false>(row, pref, counts, E, k, ids, w, ctl, debug);
+  }
 }
 
 // --------------------------------------------------------- x (bf16) staging

@@ -31,7 +31,8 @@ F_DEBUG = 8
 
 EXPORTS = ["moe_workspace_bytes", "moe_workspace_init", "moe_workspace_error", "moe_route_topk",
            "moe_expert_ffn_decode", "moe_expert_ffn_prefill", "moe_block_forward",
-           "moe_block_forward_noalloc", "moe_status_string", "moe_build_info", "moe_pack_host"]
+           "moe_block_forward_noalloc", "moe_adapt_workspace_bytes", "moe_adapt_layout",
+           "moe_status_string", "moe_build_info", "moe_pack_host"]
 
 
 class MoEError(RuntimeError):
@@ -47,7 +48,8 @@ class moe_layer(ctypes.Structure):
                 ("router_w", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
                 ("expert_slot", ctypes.c_void_p), ("codes", ctypes.c_void_p),
                 ("scales", ctypes.c_void_p), ("shared_codes", ctypes.c_void_p),
-                ("shared_scales", ctypes.c_void_p)]
+                ("shared_scales", ctypes.c_void_p), ("router_pref", ctypes.c_void_p),
+                ("route_counts", ctypes.c_void_p)]
 
 
 _lib = None
@@ -81,6 +83,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.moe_block_forward.argtypes = [P, vp, i32, vp, u32, vp, sz, vp]
     L.moe_block_forward_noalloc.restype = st
     L.moe_block_forward_noalloc.argtypes = [P, vp, i32, vp, u32, vp]
+    L.moe_adapt_workspace_bytes.restype = sz
+    L.moe_adapt_workspace_bytes.argtypes = [P, i32]
+    L.moe_adapt_layout.restype = st
+    L.moe_adapt_layout.argtypes = [P, ctypes.c_float, i32, vp, vp, sz, vp]
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_status_string.argtypes = [st]
     L.moe_build_info.restype = ctypes.c_char_p
@@ -112,12 +118,15 @@ def _check(status: int, where: str) -> None:
         raise MoEError(status, where)
 
 
-def make_layer_struct(layer) -> moe_layer:
-    """moe_layer for a ``synth.Layer`` whose tensors live on the GPU."""
+def make_layer_struct(layer, router_pref=None, route_counts=None) -> moe_layer:
+    """moe_layer for a ``synth.Layer`` whose tensors live on the GPU;
+    router_pref: optional fp32 [E] selection bonus; route_counts: optional fp32
+    [E] routing counters (both on the same device)."""
     sh = layer.shape
     return moe_layer(sh.d, sh.E, sh.F, sh.k, sh.bits, 32, sh.Fs, _ptr(layer.router_w),
                      _ptr(layer.router_bias), _ptr(layer.expert_slot), _ptr(layer.codes),
-                     _ptr(layer.scales), _ptr(layer.shared_codes), _ptr(layer.shared_scales))
+                     _ptr(layer.scales), _ptr(layer.shared_codes), _ptr(layer.shared_scales),
+                     _ptr(router_pref), _ptr(route_counts))
 
 
 def moe_workspace_bytes(layer: moe_layer, max_tokens: int) -> int:
@@ -179,6 +188,18 @@ def moe_block_forward_noalloc(layer: moe_layer, x, T: int, y, flags: int, stream
     _check(load().moe_block_forward_noalloc(ctypes.byref(layer), _ptr(x), int(T), _ptr(y),
                                             int(flags), _stream(stream)),
            "moe_block_forward_noalloc")
+
+
+def moe_adapt_workspace_bytes(layer: moe_layer, max_swaps: int) -> int:
+    return load().moe_adapt_workspace_bytes(ctypes.byref(layer), int(max_swaps))
+
+
+def moe_adapt_layout(layer: moe_layer, decay: float, max_swaps: int, swaps_done, ws, stream=None):
+    """Re-order the layer's slots by its routing counters (include/moe.h)."""
+    _check(load().moe_adapt_layout(ctypes.byref(layer), float(decay), int(max_swaps),
+                                   _ptr(swaps_done), _ptr(ws), ws.numel() * ws.element_size(),
+                                   _stream(stream)),
+           "moe_adapt_layout")
 
 
 def moe_pack_host(w, bits: int):

@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from routed_expert_ffn_06_b200 import build, moe, synth
-from _util import GpuBlock, assert_close, bf16_bits
+from _util import GpuBlock, assert_close, bf16_bits, oracle_check
 
 pytestmark = pytest.mark.gpu
 
@@ -154,3 +154,58 @@ def test_fewer_finite_logits_than_k_selects_nan_by_lowest_index():
         assert (np.sort(got[:, :3], axis=1) == np.array(finite)).all()
         nan_part = [e for e in range(SHAPE.E) if e not in finite][:7]
         assert (got[:, 3:] == np.array(nan_part)).all()
+
+
+@pytest.mark.parametrize("T", [1, 4, 8, 40])
+def test_selection_bonus_prefers_the_given_experts(T):
+    """router_pref (the pages' "router prefers experts already on the card"):
+    selection ranks logit + bonus in fp32 with the usual tie and NaN rules, the
+    weights are the softmax of the unbiased logits.  Decode-window router (T <=
+    8) and long-batch router (T = 40); the block output matches the oracle
+    selecting on the same shifted logits."""
+    wl = synth.WORKLOADS["decode"]
+    sh = wl["shape"]
+    layer = synth.make_layer(sh, seed=31, device="cuda", bias=wl["bias"], slot=wl["slot"])
+    g = torch.Generator().manual_seed(7)
+    preferred = torch.randperm(sh.E, generator=g)[:96]
+    pref = torch.zeros(sh.E, dtype=torch.float32)
+    pref[preferred] = 0.5
+    pref = pref.cuda()
+    L = moe.make_layer_struct(layer, pref)
+    ws = moe.alloc_workspace(L, max(T, 8))
+    x = synth.make_tokens(T, sh.d, seed=32, device="cuda")
+    logits = torch.empty(T, sh.E, dtype=torch.float32, device="cuda")
+    ids = torch.empty(T, sh.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, sh.k, dtype=torch.float32, device="cuda")
+    moe.moe_route_topk(L, x, T, 0, logits, ids, w, ws)
+    y = torch.empty_like(x)
+    moe.moe_block_forward(L, x, T, y, 0, ws)
+    torch.cuda.synchronize()
+    lg = logits.cpu().numpy()
+    shifted = (lg + pref.cpu().numpy()).astype(np.float32)
+    got = ids.cpu().numpy()
+    assert np.array_equal(got, oracle.select_topk_f32(shifted, sh.k))
+    assert not np.array_equal(got, oracle.select_topk_f32(lg, sh.k)), "the bonus changed nothing"
+    sel = np.take_along_axis(lg.astype(np.float64), got.astype(np.int64), axis=1)
+    own = np.exp(sel - sel.max(1, keepdims=True))
+    assert np.allclose(w.cpu().double().numpy(), own / own.sum(1, keepdims=True), rtol=1e-5, atol=1e-6)
+    r = oracle.OracleLayer(layer.to("cpu")).block_forward(bf16_bits(x), sel_logits=shifted)
+    assert np.array_equal(got, r["ids"])
+    assert_close(y, r["y"])
+
+
+@pytest.mark.parametrize("T", [1, 4, 16])
+def test_faster_mode_top_k_minus_one_full_size(T):
+    """The pages' "Faster" speed mode (5 of 6 experts, release 0.2.5) read as
+    top-(k-1): the decode layer run with top_k = 9 instead of 10 matches the
+    oracle on the decode and prefill paths."""
+    wl = synth.WORKLOADS["decode"]
+    sh = synth.MoEShape(bits=2, d=2048, E=512, F=512, Fs=512, k=9)
+    layer = synth.make_layer(sh, seed=33, device="cuda", bias=wl["bias"], slot=wl["slot"])
+    x = synth.make_tokens(T, sh.d, seed=34, device="cuda")
+    gb = GpuBlock(layer, max(T, 8))
+    logits, ids, w = gb.route(x)
+    y = gb.block(x)
+    torch.cuda.synchronize()
+    oracle_check(layer, x, logits, ids, w, y)
+    assert gb.error_word() == (0, 0)

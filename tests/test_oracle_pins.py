@@ -480,3 +480,26 @@ def test_expert_byte_counts_match_pages():
     # all experts of the model at ~2.0 bits/weight is about the "Q2_0 ~34 GB" figure
     q2 = fig["experts_total"] * per2
     assert abs(q2 / fig["q2_0_expert_bytes_total"] - 1) < 0.35
+
+
+def test_selection_bonus_reading_against_brute_force():
+    """Resident-preferring routing is read as top-k of (logit + bonus) in fp32,
+    weights from the logits alone.  With a bonus far above the logit spread on
+    a preferred set S (|S| >= k), the selection must be the top-k of S by
+    logit (ties to the lower index), and the renormalised weights the softmax
+    of those logits: checked against a brute-force sort on random rows."""
+    rng = np.random.default_rng(5)
+    E, k = 64, 10
+    for trial in range(20):
+        L = rng.standard_normal((3, E)).astype(np.float32)
+        S = np.sort(rng.choice(E, size=rng.integers(k, 30), replace=False))
+        bonus = np.zeros(E, np.float32)
+        bonus[S] = 1000.0
+        ids = oracle.select_topk_f32((L + bonus).astype(np.float32), k)
+        for t in range(3):
+            order = sorted(S, key=lambda e: (-float(L[t, e]), e))[:k]
+            assert list(ids[t]) == order
+        w = oracle.renorm_weights(L.astype(np.float64), ids)
+        sel = np.take_along_axis(L.astype(np.float64), ids.astype(np.int64), axis=1)
+        ref = np.exp(sel - sel.max(1, keepdims=True))
+        assert np.allclose(w, ref / ref.sum(1, keepdims=True), rtol=1e-12)
