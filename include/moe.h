@@ -182,8 +182,12 @@ moe_status moe_expert_ffn_prefill(const moe_layer* layer, const void* x_bf16, in
 
 /* The whole block: moe_route_topk, then the decode step for T <= 8 when the
  * layer fits the decode kernels (faster than the prefill step at every window
- * it supports) and the prefill step otherwise.  Routing lists live in the
- * workspace. */
+ * it supports) and the prefill step otherwise.  Windows of 9..32 tokens run
+ * as consecutive decode windows of up to 8 tokens (router and decode step per
+ * window), which measured faster than the prefill step there (decode layer,
+ * 2-bit: 63 vs 130 us at T = 9, 171 vs 182 us at T = 32; the prefill step
+ * wins from T = 40).  Routing lists live in the workspace; for 9..32 tokens
+ * the decode part of the workspace suffices. */
 moe_status moe_block_forward(const moe_layer* layer, const void* x_bf16, int32_t T, void* y_bf16,
                              uint32_t flags, void* ws, size_t ws_bytes, void* stream);
 

@@ -64,6 +64,9 @@ cudaError_t launch_router_large(const LayerDev& L, const uint16_t* x, int T, uin
 cudaError_t launch_router_tc(const LayerDev& L, const uint16_t* x, int T, float* logits,
                              uint16_t* hi, uint16_t* lo, Control* ctl, cudaStream_t st);
 bool decode_fits(int d, int E, int Fmax, int bits, int T);
+// Widest window the block forward runs as consecutive decode windows of up
+// to kMaxDecodeT tokens (the measured crossover to the prefill pipeline).
+constexpr int kSubWindowMaxT = 32;
 cudaError_t launch_decode(const LayerDev& L, const uint16_t* x, int T, const int32_t* ids,
                           const float* w, uint16_t* y, uint32_t flags, char* ws, const WsLayout& lay,
                           cudaStream_t st);

@@ -140,3 +140,16 @@ def test_block_forward_takes_prefill_for_experts_too_wide_for_decode(lib):
         assert full > 0
         rc = lib.moe_block_forward(ctypes.byref(L), x, 4, y, 0, 0x7F0000600000, full - 1, None)
         assert rc == want, (ffn, rc)
+
+
+def test_block_forward_middle_windows_need_only_the_decode_workspace(lib):
+    """Windows of 9..32 tokens run as consecutive decode windows, which need
+    only the decode part of the workspace (one byte short of the full size
+    passes and stops at the missing device); 33 tokens take the prefill step
+    and need it all."""
+    x, y = 0x7F0000400000, 0x7F0000500000
+    L = _layer(d_model=256, n_experts=20, ffn=512, shared_ffn=512, top_k=16)
+    for T, want in [(9, 8), (16, 8), (32, 8), (33, 3)]:
+        full = lib.moe_workspace_bytes(ctypes.byref(L), T)
+        rc = lib.moe_block_forward(ctypes.byref(L), x, T, y, 0, 0x7F0000600000, full - 1, None)
+        assert rc == want, (T, rc)

@@ -213,3 +213,28 @@ def test_block_forward_uses_decode_up_to_eight_tokens(T):
     torch.cuda.synchronize()
     assert torch.equal(y, yd)
     oracle_check(layer, x, logits, ids, w, y)
+
+
+@pytest.mark.parametrize("T", [9, 16, 33, 64])
+def test_block_forward_middle_windows(T):
+    """Windows wider than the decode kernels: 9..32 tokens run as consecutive
+    decode windows of up to 8 tokens (the measured crossover), wider ones on
+    the prefill step.  Routing and outputs match the oracle; up to 32 tokens
+    the output equals the explicit 8-token decode calls byte for byte."""
+    wl = synth.WORKLOADS["decode"]
+    layer = synth.make_layer(wl["shape"], seed=8, device="cuda", bias=wl["bias"], slot=wl["slot"])
+    x = synth.make_tokens(T, 2048, seed=60 + T, device="cuda")
+    gb = GpuBlock(layer, T)
+    logits, ids, w = gb.route(x)
+    y = gb.block(x)
+    torch.cuda.synchronize()
+    oracle_check(layer, x, logits, ids, w, y)
+    if T <= 32:
+        parts = []
+        for t0 in range(0, T, 8):
+            xs = x[t0:t0 + 8].clone()
+            _, i8, w8 = gb.route(xs)
+            parts.append(gb.decode(xs, i8, w8))
+        torch.cuda.synchronize()
+        assert torch.equal(y, torch.cat(parts))
+    assert gb.error_word() == (0, 0)
