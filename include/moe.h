@@ -143,6 +143,36 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * MOE_ERR_TIMEOUT / MOE_ERR_DEVICE_CHECK when the word was set. */
 moe_status moe_workspace_error(void* ws, size_t ws_bytes, uint32_t* code_out, void* stream);
 
+/* Set the limit of the kernels' bounded waits for calls on this workspace
+ * (enqueued on stream; a one-thread kernel, so it may be graph-captured).
+ * Every wait of a kernel on a pipeline barrier (a shared-memory stage, a
+ * tensor-memory accumulator, an asynchronous copy) gives up after limit_us
+ * microseconds of the GPU's global timer, records MOE_ERR_TIMEOUT in the
+ * error word and stops issuing work; before its thread block ends it waits
+ * for the copies and tensor-core operations it already issued.  The outputs of
+ * a call that timed out are undefined; the workspace stays usable.
+ * limit_us = 0 restores the default of one second; other values from 1,000
+ * (1 ms: a wait reads the limit only once it has lasted that long) to
+ * 60,000,000 (60 s), else MOE_ERR_INVALID_ARG.  moe_workspace_init() restores the default.  The
+ * pages' engine has no counterpart: this bounds a stuck pipeline. */
+moe_status moe_workspace_set_wait_limit(void* ws, size_t ws_bytes, uint32_t limit_us, void* stream);
+
+/* Test switch for the bounded-wait path (enqueued on stream like the call
+ * above).  site = 1: in calls that pass MOE_F_DEBUG and run the prefill
+ * expert step (moe_expert_ffn_prefill, or moe_block_forward with T > 32), one
+ * epilogue thread of thread block 0 of the gate/up GEMM skips its plain
+ * arrive on the barrier that frees the first tensor-memory accumulator, so
+ * the MMA issuer's wait before that block's third work item runs out (a call
+ * with at least 3 x 148 gate/up work items, e.g. 64 tokens of a 512-expert
+ * layer, reaches it) and the call ends with MOE_ERR_TIMEOUT in the error word
+ * after a few wait limits; the copies and MMAs already issued complete
+ * before the thread block ends.  Calls without MOE_F_DEBUG ignore the
+ * switch.  site = 0 turns it off; other values return
+ * MOE_ERR_INVALID_ARG.  moe_workspace_init() turns it off.  No counterpart
+ * in the pages: it exists to test the error path without a fault. */
+moe_status moe_workspace_set_debug_withhold(void* ws, size_t ws_bytes, uint32_t site,
+                                            void* stream);
+
 /* Router + top-k + softmax renormalisation for T tokens.
  *  x_bf16: dev bf16 [T][d].  flags: MOE_F_PRENORM and MOE_F_DEBUG honoured.
  *  logits_or_null: dev fp32 [T][E], written when non-NULL.

@@ -18,17 +18,25 @@ constexpr uint32_t kErrTimeout = 1u;      // a bounded wait ran out
 constexpr uint32_t kErrRange = 2u;        // an id / slot / size outside its range
 constexpr uint32_t kErrNonFinite = 4u;    // a non-finite value where finite is required
 
-// Bounded waits give up after this many nanoseconds of %globaltimer.
+// Bounded waits give up after this many nanoseconds of %globaltimer, unless
+// the control block carries a limit of its own.
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+
+// Test switch (control block word debug_withhold, honoured only under
+// MOE_F_DEBUG): thread 0 of CTA 0 of the prefill gate/up GEMM's epilogue skips
+// its plain arrive on the first accumulator's "TMEM free" barrier, so that the
+// MMA issuer's wait before the CTA's third work item runs out.
+constexpr uint32_t kWithholdPrefillArrive = 1u;
 
 // Workspace control block (first 256 bytes of every workspace).
 struct Control {
   uint32_t err;            // OR of kErr* bits
   uint32_t router_done;    // CTAs of the small-T router that finished (self-resetting)
   uint32_t prefill_done;   // CTAs of the prefill bucketing pass that finished (self-resetting)
-  uint32_t pad0;
+  uint32_t wait_limit_us;  // bounded-wait limit in microseconds; 0: kWaitLimitNs
   uint32_t err_where;      // first failing site (debug aid)
-  uint32_t pad[59];
+  uint32_t debug_withhold; // test switch (kWithhold*), 0: off
+  uint32_t pad[58];
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 
@@ -97,17 +105,29 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; gives up after
-// kWaitLimitNs of %globaltimer, records kErrTimeout and returns false.
+// Wait for the phase with the given parity to complete; gives up after the
+// control block's limit (kWaitLimitNs when it holds 0) of %globaltimer,
+// records kErrTimeout and returns false.  The limit is read only once a wait
+// has lasted kWaitFloorNs, so the waits of a running pipeline never load it;
+// limits below the floor are not accepted by the host.
+constexpr unsigned long long kWaitFloorNs = 1000000ull;   // 1 ms
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Control* ctl,
                                           uint32_t where) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
+  unsigned long long limit = 0;   // not read yet
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      record_error(ctl, kErrTimeout, where);
-      return false;
+    const unsigned long long el = globaltimer_ns() - t0;
+    if (el > kWaitFloorNs) {
+      if (limit == 0) {
+        const uint32_t us = ctl ? *reinterpret_cast<volatile uint32_t*>(&ctl->wait_limit_us) : 0u;
+        limit = us ? 1000ull * us : kWaitLimitNs;
+      }
+      if (el > limit) {
+        record_error(ctl, kErrTimeout, where);
+        return false;
+      }
     }
   }
 }
@@ -179,6 +199,21 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Named barrier over `count` threads (multiple of 32).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier over `count` threads that also returns whether any of them
+// passed pred = true (every participant gets the same answer).
+__device__ __forceinline__ bool named_bar_any(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 }  // namespace moe

@@ -94,6 +94,14 @@ moe_status from_cuda(cudaError_t e) {
   return MOE_ERR_CUDA;
 }
 
+__global__ void set_word_kernel(uint32_t* p, uint32_t v) { *p = v; }
+
+// One word of a workspace control block, written in stream order.
+moe_status set_control_word(uint32_t* p, uint32_t v, cudaStream_t st) {
+  set_word_kernel<<<1, 1, 0, st>>>(p, v);
+  return from_cuda(cudaGetLastError());
+}
+
 // Common preamble of every compute entry point.
 moe_status preamble(const moe_layer* layer, int32_t T, const void* x, void* ws, size_t ws_bytes,
                     bool decode_path,
@@ -259,6 +267,29 @@ moe_status moe_workspace_error(void* ws, size_t ws_bytes, uint32_t* code_out, vo
   if (code & kErrTimeout) return MOE_ERR_TIMEOUT;
   if (code) return MOE_ERR_DEVICE_CHECK;
   return MOE_OK;
+}
+
+moe_status moe_workspace_set_wait_limit(void* ws, size_t ws_bytes, uint32_t limit_us,
+                                        void* stream) {
+  if (!ws || ws_bytes < sizeof(Control) || limit_us > 60000000u ||
+      (limit_us != 0 && limit_us < kWaitFloorNs / 1000))
+    return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MOE_ERR_MISALIGNED;
+  moe_status s = check_device();
+  if (s != MOE_OK) return s;
+  return set_control_word(&static_cast<Control*>(ws)->wait_limit_us, limit_us,
+                          static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_workspace_set_debug_withhold(void* ws, size_t ws_bytes, uint32_t site,
+                                            void* stream) {
+  if (!ws || ws_bytes < sizeof(Control) || site > kWithholdPrefillArrive)
+    return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MOE_ERR_MISALIGNED;
+  moe_status s = check_device();
+  if (s != MOE_OK) return s;
+  return set_control_word(&static_cast<Control*>(ws)->debug_withhold, site,
+                          static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_route_topk(const moe_layer* layer, const void* x_bf16, int32_t T, uint32_t flags,

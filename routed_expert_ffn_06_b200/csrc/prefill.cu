@@ -331,6 +331,7 @@ struct PfArgs {
   int T;
   int Fmax;
   int ppc;      // tile pairs (work items) per chunk
+  int debug;    // MOE_F_DEBUG given: the control block's test switch is honoured
   PfWs p;
   Control* ctl;
 };
@@ -651,7 +652,7 @@ __host__ __device__ inline PfSmem pf_smem() {
   m.out = o;                       // epilogue staging: two 32-row blocks
   o += 2 * (size_t)PF_OUT_STAGE;
   m.bars = o;
-  o += (2 * PF_NS + 4) * 8;
+  o += (3 * PF_NS + 5) * 8;
   m.holder = o;
   o += 16;
   m.total = o + 1024;   // slack to align the base to 1024
@@ -668,23 +669,27 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
   unsigned char* sA = smem + m.a;
   unsigned char* sB = smem + m.b;
   unsigned char* sOut = smem + m.out;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + m.bars);   // A by 4 warps + B by TMA
-  uint64_t* empty = full + PF_NS;                                  // MMA commit
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + m.bars);   // A: 4 producer warps
+  uint64_t* bfull = full + PF_NS;                                  // B: the TMA load
+  uint64_t* empty = bfull + PF_NS;                                 // MMA commit
   uint64_t* tfull = empty + PF_NS;
   uint64_t* tempty = tfull + 2;
+  uint64_t* mdone = tempty + 2;                                    // every MMA issued has completed
   uint32_t* holder = reinterpret_cast<uint32_t*>(smem + m.holder);
   Control* ctl = a.ctl;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     for (int s = 0; s < PF_NS; ++s) {
-      mbar_init(&full[s], PF_A_WARPS + 1);
+      mbar_init(&full[s], PF_A_WARPS);
+      mbar_init(&bfull[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 128);
     }
+    mbar_init(mdone, 1);
     fence_barrier_init();
   }
   if (warp == 12) {
@@ -701,6 +706,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
   tc_fence_after();
   const uint32_t tmem_base = *holder;
   const int n_items = a.p.misc[0] * a.ppc;
+  // Give-up rule: a role whose bounded wait runs out (the timeout is recorded
+  // in the error word) stops issuing copies, MMAs, stores and arrives, and
+  // leaves its loop; the decision is uniform over the warp (over the four
+  // epilogue warps for the epilogue).  Before the CTA releases its TMEM and
+  // shared memory, the loader waits for every copy it issued and the MMA
+  // issuer for every MMA it issued, so nothing asynchronous is in flight when
+  // the CTA ends.  The roles left waiting on a role that gave up run out in
+  // turn, so a stuck pipeline ends within a few wait limits.
   bool ok = true;
 
   if (warp >= 4 && warp < 12) {
@@ -720,9 +733,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
     q.init(a, n_items);
     if (grp == 1 && !q.done) q.advance(a);
     // Rotating register buffers: no copy of a buffer ever waits on its loads.
-    auto produce = [&](const PfRaw& r, int g) {
+    // Returns false when the wait for the stage ran out.
+    auto produce = [&](const PfRaw& r, int g) -> bool {
       const int sa = g % PF_NS;
-      if (g >= PF_NS && ok) ok = mbar_wait(&empty[sa], ((g / PF_NS) - 1) & 1, ctl, 0x611);
+      if (g >= PF_NS) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&empty[sa], ((g / PF_NS) - 1) & 1, ctl, 0x611));
+        if (!ok) return false;
+      }
       if (gi < (int)(r.meta >> 4)) {
         // unit u: tile u >> 1 (+16 KB), row rq + 64 (u & 1) (+8 KB); absent
         // units (rows outside the matrix) are written as zeros
@@ -745,6 +762,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[sa]);
+      return true;
     };
     auto skip2 = [&]() {   // this group's next k-step
       q.advance(a);
@@ -774,7 +792,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
         pf_load_raw<BITS>(a, q, rq, gi, U, r2);
         skip2();
       }
-      produce(r0, g);
+      if (!produce(r0, g)) break;
       g += 2;
       if (!h1) break;
       h0 = !q.done;
@@ -782,7 +800,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
         pf_load_raw<BITS>(a, q, rq, gi, U, r0);
         skip2();
       }
-      produce(r1, g);
+      if (!produce(r1, g)) break;
       g += 2;
       if (!h2) break;
       h1 = !q.done;
@@ -790,7 +808,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
         pf_load_raw<BITS>(a, q, rq, gi, U, r1);
         skip2();
       }
-      produce(r2, g);
+      if (!produce(r2, g)) break;
       g += 2;
     }
   } else if (warp == 13) {
@@ -812,10 +830,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
         if (leader) pf_prefetch_item<BITS>(a, pit);
         have = pfs.get(a, pit);
       }
-      if (g >= PF_NS && ok) ok = mbar_wait(&empty[sb], pb ^ 1u, ctl, 0x620);
+      if (g >= PF_NS) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&empty[sb], pb ^ 1u, ctl, 0x620));
+        if (!ok) break;
+      }
       if (leader) {
-        mbar_arrive_expect_tx(&full[sb], PF_B_STAGE);
-        tma_load_2d(sB + sb * PF_B_STAGE, &mp.b, 64 * cur.ks, cur.item_ref().pos0, &full[sb]);
+        mbar_arrive_expect_tx(&bfull[sb], PF_B_STAGE);
+        tma_load_2d(sB + sb * PF_B_STAGE, &mp.b, 64 * cur.ks, cur.item_ref().pos0, &bfull[sb]);
       }
       __syncwarp();
       if (++sb == PF_NS) {
@@ -825,6 +846,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
       cur.advance(a);
       ++g;
     }
+    // The last min(g, PF_NS) copies, one per stage and each its stage's newest
+    // phase, may not have been consumed (always the case after a give-up
+    // anywhere in the CTA): wait for them to land.  On the normal path they
+    // have landed already.
+    if (leader)
+      for (int j = g > PF_NS ? g - PF_NS : 0; j < g; ++j)
+        mbar_wait(&bfull[j % PF_NS], (uint32_t)(j / PF_NS) & 1u, ctl, 0x621);
+    __syncwarp();
   } else if (warp == 12) {
     // ------------------------------------------------ MMA issuer
     // The whole warp walks the loop (its values stay warp-uniform); one
@@ -837,48 +866,63 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
     PfItem it;
     int s = 0, la = 0;
     uint32_t ph = 0;
+    bool issued = false;
     while (seq.get(a, it)) {
       const int acc = la & 1;
-      if (la >= 2 && ok) ok = mbar_wait(&tempty[acc], ((la >> 1) - 1) & 1, ctl, 0x630);
+      if (la >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&tempty[acc], ((la >> 1) - 1) & 1, ctl, 0x630));
+        if (!ok) break;
+      }
       tc_fence_after();
       const uint32_t idesc = idesc_f16_f32(PF_BM, (it.nv + 15) & ~15);
       const uint32_t d0 = tmem_base + (uint32_t)(acc * 256), d1 = d0 + 128;
       const bool two = it.two;
       for (int ks = 0; ks < it.KS; ++ks) {
-        if (ok) ok = mbar_wait(&full[s], ph, ctl, 0x631);
+        // B (one TMA load) lands long before the dequantised A tile: its
+        // wait is passed by the time A's completes
+        bool got = mbar_wait(&bfull[s], ph, ctl, 0x632);
+        got = got && mbar_wait(&full[s], ph, ctl, 0x631);
+        ok = __all_sync(0xffffffffu, got);
+        if (!ok) break;
         tc_fence_after();
         const uint64_t ad = adesc0 + (uint64_t)(s * (PF_A_STAGE >> 4));
         const uint64_t bd = bdesc0 + (uint64_t)(s * (PF_B_STAGE >> 4));
         const uint32_t first = ks > 0 ? 1u : 0u;
         const bool full = ks < it.KS - 1 || it.ng_last == 2;
         if (leader) {
-          if (ok) {
-            tc_mma_f16(d0, ad, bd, idesc, first);
-            tc_mma_f16(d0, ad + 2, bd + 2, idesc, 1u);
+          tc_mma_f16(d0, ad, bd, idesc, first);
+          tc_mma_f16(d0, ad + 2, bd + 2, idesc, 1u);
+          if (two) {
+            tc_mma_f16(d1, ad + (PF_A_TILE >> 4), bd, idesc, first);
+            tc_mma_f16(d1, ad + (PF_A_TILE >> 4) + 2, bd + 2, idesc, 1u);
+          }
+          if (full) {
+            tc_mma_f16(d0, ad + 4, bd + 4, idesc, 1u);
+            tc_mma_f16(d0, ad + 6, bd + 6, idesc, 1u);
             if (two) {
-              tc_mma_f16(d1, ad + (PF_A_TILE >> 4), bd, idesc, first);
-              tc_mma_f16(d1, ad + (PF_A_TILE >> 4) + 2, bd + 2, idesc, 1u);
-            }
-            if (full) {
-              tc_mma_f16(d0, ad + 4, bd + 4, idesc, 1u);
-              tc_mma_f16(d0, ad + 6, bd + 6, idesc, 1u);
-              if (two) {
-                tc_mma_f16(d1, ad + (PF_A_TILE >> 4) + 4, bd + 4, idesc, 1u);
-                tc_mma_f16(d1, ad + (PF_A_TILE >> 4) + 6, bd + 6, idesc, 1u);
-              }
+              tc_mma_f16(d1, ad + (PF_A_TILE >> 4) + 4, bd + 4, idesc, 1u);
+              tc_mma_f16(d1, ad + (PF_A_TILE >> 4) + 6, bd + 6, idesc, 1u);
             }
           }
           tc_commit(&empty[s]);
         }
+        issued = true;
         __syncwarp();
         if (++s == PF_NS) {
           s = 0;
           ph ^= 1u;
         }
       }
+      if (!ok) break;
       if (leader) tc_commit(&tfull[acc]);
       __syncwarp();
       ++la;
+    }
+    // every MMA issued has completed before the CTA releases its TMEM
+    if (issued) {
+      if (leader) tc_commit(mdone);
+      __syncwarp();
+      mbar_wait(mdone, 0, ctl, 0x633);
     }
   } else {
     // ------------------------------------------------ epilogue (warps 0-3)
@@ -890,6 +934,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
     seq.init(a, n_items);
     PfItem it;
     int la = 0, cc = 0;
+    // test switch: thread 0 of block 0 of the gate/up GEMM keeps back its
+    // arrive on the first accumulator's barrier, so the MMA issuer's wait
+    // before its third item runs out (held here, not in the producer warps,
+    // which are the pipeline's bottleneck)
+    const bool withhold =
+        a.debug && a.mode == 0 && blockIdx.x == 0 && tid == 0 &&
+        *reinterpret_cast<volatile uint32_t*>(&ctl->debug_withhold) == kWithholdPrefillArrive;
     // free a staging buffer (the store issued from it two blocks ago has read it)
     auto claim = [&]() {
       if (tid == 0 && cc >= 2) bulk_wait_read<1>();
@@ -913,7 +964,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
         for (int c = 0; c < 4; ++c)
           if (lane + 32 * c < it.nv) wcol[c] = a.p.wpos[it.pos0 + lane + 32 * c];
       }
-      if (ok) ok = mbar_wait(&tfull[acc], (la >> 1) & 1, ctl, 0x640);
+      ok = mbar_wait(&tfull[acc], (la >> 1) & 1, ctl, 0x640);
+      if (named_bar_any(3, 128, !ok)) {   // one epilogue thread gave up: all four warps stop
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const int n_mma = (it.nv + 15) & ~15;
       const int ntile = it.two ? 2 : 1;
@@ -926,7 +981,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
           tmem_ld_wait();
           if (v == ntile - 1 && c0 + 32 >= n_mma) {
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);   // TMEM free: the MMA may start item + 2
+            if (!(withhold && la == 0)) mbar_arrive(&tempty[acc]);   // TMEM free: item + 2 may start
           }
           claim();
           __half* so = reinterpret_cast<__half*>(sOut + (cc & 1) * PF_OUT_STAGE);
@@ -1115,6 +1170,7 @@ cudaError_t launch_prefill(const LayerDev& L, const uint16_t* x, int T, const in
   a.Fmax = Fmax;
   a.p = p;
   a.ctl = ctl;
+  a.debug = (flags & MOE_F_DEBUG) ? 1 : 0;
   a.mode = 0;
   a.ppc = (Fmax + 127) / 128;
   e = L.bits == 2 ? launch_gemm<2>(a, m0, st) : launch_gemm<3>(a, m0, st);

@@ -98,12 +98,14 @@ __global__ void __launch_bounds__(RT_THREADS, 1) router_tc_kernel(const float* _
   const uint32_t tmem = *holder;
   bool ok = true;
 
+  // A role whose bounded wait runs out stops issuing; before the CTA ends, the
+  // loader waits for the copies it issued and the MMA lane for its MMAs.
   if (warp == 0) {
     if (lane == 0) {
-      int s = 0;
+      int s = 0, ks = 0;
       uint32_t ph = 0;
-      for (int ks = 0; ks < KS; ++ks) {
-        if (ks >= RT_STAGES && ok) ok = mbar_wait(&empty[s], ph ^ 1u, ctl, 0x250);
+      for (; ks < KS; ++ks) {
+        if (ks >= RT_STAGES && !mbar_wait(&empty[s], ph ^ 1u, ctl, 0x250)) break;
         unsigned char* st = smem + s * RT_STAGE;
         mbar_arrive_expect_tx(&full[s], RT_STAGE);
         rt_tma_2d(st, &mp.hi, 64 * ks, e0, &full[s]);
@@ -114,6 +116,9 @@ __global__ void __launch_bounds__(RT_THREADS, 1) router_tc_kernel(const float* _
           ph ^= 1u;
         }
       }
+      // the newest phase of each stage may be unconsumed: its copies land first
+      for (int j = ks > RT_STAGES ? ks - RT_STAGES : 0; j < ks; ++j)
+        mbar_wait(&full[j % RT_STAGES], (uint32_t)(j / RT_STAGES) & 1u, ctl, 0x253);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -123,27 +128,28 @@ __global__ void __launch_bounds__(RT_THREADS, 1) router_tc_kernel(const float* _
       int s = 0;
       uint32_t ph = 0;
       for (int ks = 0; ks < KS; ++ks) {
-        if (ok) ok = mbar_wait(&full[s], ph, ctl, 0x251);
+        if (!mbar_wait(&full[s], ph, ctl, 0x251)) break;
         tc_fence_after();
         const uint64_t ah = desc0 + (uint64_t)(s * (RT_STAGE >> 4));
         const uint64_t al = ah + (RT_TILE >> 4), bx = ah + 2 * (RT_TILE >> 4);
-        if (ok) {
-          tc_mma_f16(tmem, ah, bx, idesc, ks > 0 ? 1u : 0u);
-          tc_mma_f16(tmem, ah + 2, bx + 2, idesc, 1u);
-          tc_mma_f16(tmem, ah + 4, bx + 4, idesc, 1u);
-          tc_mma_f16(tmem, ah + 6, bx + 6, idesc, 1u);
-          tc_mma_f16(tmem, al, bx, idesc, 1u);
-          tc_mma_f16(tmem, al + 2, bx + 2, idesc, 1u);
-          tc_mma_f16(tmem, al + 4, bx + 4, idesc, 1u);
-          tc_mma_f16(tmem, al + 6, bx + 6, idesc, 1u);
-        }
+        tc_mma_f16(tmem, ah, bx, idesc, ks > 0 ? 1u : 0u);
+        tc_mma_f16(tmem, ah + 2, bx + 2, idesc, 1u);
+        tc_mma_f16(tmem, ah + 4, bx + 4, idesc, 1u);
+        tc_mma_f16(tmem, ah + 6, bx + 6, idesc, 1u);
+        tc_mma_f16(tmem, al, bx, idesc, 1u);
+        tc_mma_f16(tmem, al + 2, bx + 2, idesc, 1u);
+        tc_mma_f16(tmem, al + 4, bx + 4, idesc, 1u);
+        tc_mma_f16(tmem, al + 6, bx + 6, idesc, 1u);
         tc_commit(&empty[s]);
         if (++s == RT_STAGES) {
           s = 0;
           ph ^= 1u;
         }
       }
+      // done arrives once every MMA issued has completed (also after a
+      // give-up); this lane releases the TMEM only after that
       tc_commit(done);
+      mbar_wait(done, 0, ctl, 0x254);
     }
   } else {
     // epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 = experts of those rows

@@ -29,7 +29,11 @@ F_RESIDUAL = 2
 F_DETERMINISTIC = 4
 F_DEBUG = 8
 
-EXPORTS = ["moe_workspace_bytes", "moe_workspace_init", "moe_workspace_error", "moe_route_topk",
+# moe_workspace_set_debug_withhold sites
+WITHHOLD_PREFILL_ARRIVE = 1
+
+EXPORTS = ["moe_workspace_bytes", "moe_workspace_init", "moe_workspace_error",
+           "moe_workspace_set_wait_limit", "moe_workspace_set_debug_withhold", "moe_route_topk",
            "moe_expert_ffn_decode", "moe_expert_ffn_prefill", "moe_block_forward",
            "moe_block_forward_noalloc", "moe_adapt_workspace_bytes", "moe_adapt_layout",
            "moe_status_string", "moe_build_info", "moe_pack_host"]
@@ -73,6 +77,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.moe_workspace_init.argtypes = [vp, sz, vp]
     L.moe_workspace_error.restype = st
     L.moe_workspace_error.argtypes = [vp, sz, ctypes.POINTER(u32), vp]
+    L.moe_workspace_set_wait_limit.restype = st
+    L.moe_workspace_set_wait_limit.argtypes = [vp, sz, u32, vp]
+    L.moe_workspace_set_debug_withhold.restype = st
+    L.moe_workspace_set_debug_withhold.argtypes = [vp, sz, u32, vp]
     L.moe_route_topk.restype = st
     L.moe_route_topk.argtypes = [P, vp, i32, u32, vp, vp, vp, vp, sz, vp]
     L.moe_expert_ffn_decode.restype = st
@@ -143,6 +151,18 @@ def moe_workspace_error(ws: torch.Tensor, stream=None):
     st = load().moe_workspace_error(_ptr(ws), ws.numel() * ws.element_size(), ctypes.byref(code),
                                     _stream(stream))
     return st, code.value
+
+
+def moe_workspace_set_wait_limit(ws: torch.Tensor, limit_us: int, stream=None) -> None:
+    _check(load().moe_workspace_set_wait_limit(_ptr(ws), ws.numel() * ws.element_size(),
+                                               int(limit_us), _stream(stream)),
+           "moe_workspace_set_wait_limit")
+
+
+def moe_workspace_set_debug_withhold(ws: torch.Tensor, site: int, stream=None) -> None:
+    _check(load().moe_workspace_set_debug_withhold(_ptr(ws), ws.numel() * ws.element_size(),
+                                                   int(site), _stream(stream)),
+           "moe_workspace_set_debug_withhold")
 
 
 def alloc_workspace(layer: moe_layer, max_tokens: int, device=None) -> torch.Tensor:

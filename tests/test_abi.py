@@ -153,3 +153,23 @@ def test_block_forward_middle_windows_need_only_the_decode_workspace(lib):
         full = lib.moe_workspace_bytes(ctypes.byref(L), T)
         rc = lib.moe_block_forward(ctypes.byref(L), x, T, y, 0, 0x7F0000600000, full - 1, None)
         assert rc == want, (T, rc)
+
+
+def test_wait_limit_and_withhold_switch_validation(lib):
+    """The control-block setters check their arguments on the host; valid
+    calls stop at the missing device."""
+    ws = 0x7F0000600000
+    set_limit, set_site = lib.moe_workspace_set_wait_limit, lib.moe_workspace_set_debug_withhold
+    assert set_limit(None, 1 << 20, 1000, None) == 1
+    assert set_limit(ws, 64, 1000, None) == 1                  # smaller than the control block
+    assert set_limit(ws + 16, 1 << 20, 1000, None) == 4        # not 256-aligned
+    assert set_limit(ws, 1 << 20, 60_000_001, None) == 1       # above 60 s
+    assert set_limit(ws, 1 << 20, 999, None) == 1              # below the 1 ms floor
+    assert set_site(ws, 1 << 20, 2, None) == 1                 # no such site
+    assert set_site(None, 1 << 20, 1, None) == 1
+    assert set_site(ws + 16, 1 << 20, 1, None) == 4
+    import torch
+    if not torch.cuda.is_available():
+        assert set_limit(ws, 1 << 20, 60_000_000, None) == 8
+        assert set_limit(ws, 1 << 20, 0, None) == 8
+        assert set_site(ws, 1 << 20, moe.WITHHOLD_PREFILL_ARRIVE, None) == 8
