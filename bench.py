@@ -57,6 +57,9 @@ def parse():
     p.add_argument("--adapt-decay", type=float, default=0.5)
     p.add_argument("--rounds", type=int, default=2048,
                    help="rounds of the T=1..4 windows in one decode step (smaller for profiling)")
+    p.add_argument("--no-l2-next", dest="l2_next", action="store_false",
+                   help="do not let each decode step prefetch the next layer's router and shared "
+                        "expert into L2")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-prefill", action="store_true",
                    help="decode workload only (no prefill object in the line)")
@@ -265,6 +268,8 @@ def bench_decode(args, rank, world, local):
         prefs = [torch.where(l.rank.to(dev) <= args.prefer_hot, args.prefer_bonus, 0.0).float()
                  for l in layers]
     structs = [moe.make_layer_struct(l, p) for l, p in zip(layers, prefs)]
+    if args.l2_next:   # window w runs on copy w % NL: its successor is the next copy
+        moe.link_l2_next(structs)
     ws = moe.alloc_workspace(structs[0], max(DECODE_WINDOWS))
     # fresh tokens for every window of a step
     xs = [[synth.make_tokens(T, sh.d, seed=rank * 1000 + 7, step=r * nwin + i, device=dev)
@@ -417,6 +422,7 @@ def bench_decode(args, rank, world, local):
                    "parallelism": f"replicas x{world}",
                    "mma": "f16 x f16 -> f32 (weights dequantised in registers)",
                    "unique_experts_per_window": U_mean, "zipf_s_fitted": round(zipf_s, 3),
+                   "l2_prefetch_next": bool(args.l2_next),
                    "top_k": sh.k, "prefer_hot": args.prefer_hot,
                    "prefer_bonus": args.prefer_bonus if args.prefer_hot else None,
                    "weights_gen_s": round(t_gen, 1)},
@@ -644,6 +650,8 @@ def bench_stack(args, rank, world, local):
     layers = _stack_layers(wl, rank, dev)
     t_gen = time.time() - t_gen
     structs = [moe.make_layer_struct(l) for l in layers]
+    if args.l2_next:   # layer l is followed by l + 1, the last by the next step's first
+        moe.link_l2_next(structs)
     ws = moe.alloc_workspace(structs[0], T)
     G = 16
     x0 = [synth.make_tokens(T, sh.d, seed=rank * 1000 + 9, step=s, device=dev) for s in range(G)]
@@ -721,6 +729,7 @@ def bench_stack(args, rank, world, local):
                    "tokens_per_step": T,
                    "weights_gb": round(NLy * (sh.E * eb + eb + sh.E * sh.d * 4) / 1e9, 2),
                    "l2": "inputs larger than L2 (34 GB of weights per step)",
+                   "l2_prefetch_next": bool(args.l2_next),
                    "weights_gen_s": round(t_gen, 1), "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -759,6 +768,8 @@ def bench_mix(args, rank, world, local):
     AE = args.adapt_every
     counts = [torch.zeros(sh.E, dtype=torch.float32, device=dev) if AE else None for _ in layers]
     structs = [moe.make_layer_struct(l, route_counts=c) for l, c in zip(layers, counts)]
+    if args.l2_next:
+        moe.link_l2_next(structs)
     ws = moe.alloc_workspace(structs[0], C)
     if AE:
         n = moe.moe_adapt_workspace_bytes(structs[0], args.adapt_swaps)
@@ -834,6 +845,7 @@ def bench_mix(args, rank, world, local):
                                "512 decode steps of 4 tokens, expert ranking re-drawn every 64 steps",
                    "tokens": ntok, "weights_gb": round(NLy * (sh.E * eb + eb + sh.E * sh.d * 4) / 1e9, 2),
                    "l2": "inputs larger than L2 (34 GB of weights)",
+                   "l2_prefetch_next": bool(args.l2_next),
                    "weights_gen_s": round(t_gen, 1), "parallelism": f"replicas x{world}"},
         "adaptive_layout": ({"every_steps": AE, "max_swaps": args.adapt_swaps,
                              "decay": args.adapt_decay} if AE else None),

@@ -96,7 +96,7 @@ typedef enum {
 #define MOE_F_DEBUG 8u          /* kernels range-check ids, slots and values */
 
 /* One layer.  A host struct, read only during the call. */
-typedef struct {
+typedef struct moe_layer_s {
   int32_t d_model;       /* d */
   int32_t n_experts;     /* E */
   int32_t ffn;           /* F, routed experts' hidden size */
@@ -126,6 +126,18 @@ typedef struct {
    * exact below 2^24); moe_adapt_layout reads and decays them.  Selections
    * passed in by the caller (the expert-step calls) are not counted. */
   float* route_counts;
+  /* host pointer or NULL: the layer the caller runs after this one.  Its
+   * input-independent weights (router_w, shared_codes, shared_scales) are
+   * prefetched into L2 (cp.async.bulk.prefetch.L2, spread over the thread
+   * blocks) by this layer's decode expert step, so that the next layer's
+   * router and shared expert read them from L2 instead of HBM.  A hint: the
+   * results do not depend on it.  Read during the call like this struct; its
+   * shape fields must pass the limits above and its pointers be 16-byte
+   * aligned, else the call returns MOE_ERR_INVALID_ARG.  The pages overlap
+   * the next layer's weight transfer with the current layer's compute in the
+   * same way ("Strata illustrated", section on long prompts: the next
+   * layer's experts stream in while the current layer computes). */
+  const struct moe_layer_s* l2_next;
 } moe_layer;
 
 /* Bytes of workspace the calls below need for up to max_tokens tokens

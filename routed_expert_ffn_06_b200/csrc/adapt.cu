@@ -155,7 +155,7 @@ using namespace moe;
 extern "C" size_t moe_adapt_workspace_bytes(const moe_layer* layer, int32_t max_swaps) {
   if (!layer || max_swaps < 0 || layer->n_experts < 1 || layer->n_experts > 1024) return 0;
   if (moe_workspace_bytes(layer, 1) == 0) return 0;   // the layer checks
-  LayerDev L;
+  LayerDev L{};
   L.d = layer->d_model;
   L.F = layer->ffn;
   L.E = layer->n_experts;
@@ -176,7 +176,7 @@ extern "C" moe_status moe_adapt_layout(const moe_layer* layer, float decay, int3
   if (!layer->codes || !layer->scales || !layer->expert_slot) return MOE_ERR_INVALID_ARG;
   moe_status s = check_device();
   if (s != MOE_OK) return s;
-  LayerDev L;
+  LayerDev L{};
   L.d = layer->d_model;
   L.E = layer->n_experts;
   L.F = layer->ffn;

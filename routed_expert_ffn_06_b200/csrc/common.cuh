@@ -144,6 +144,11 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32
       : "memory");
 }
 
+// Hint: bring [src, src + bytes) into L2.  16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------ programmatic dependent launch
 // griddepcontrol.wait: block until the grids this one depends on completed and
 // their memory is visible (a no-op when launched without the PDL attribute).

@@ -377,6 +377,17 @@ __global__ void __launch_bounds__(kGuWarps * 32, 1)
     for (int s = 0; s < kGuWarps * spw; ++s) mbar_init(&bars[s], 1);
     fence_barrier_init();
   }
+  if (tid == 32) {
+    // the next layer's router and shared expert into L2: an equal 16-byte
+    // aligned slice of each range per CTA (constant data, so before the wait)
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+      const unsigned B = L.pfb[r];
+      const unsigned chunk = ((B + gridDim.x - 1) / gridDim.x + 15u) & ~15u;
+      const unsigned lo = chunk * blockIdx.x;
+      if (lo < B) prefetch_l2(L.pf[r] + lo, B - lo < chunk ? B - lo : chunk);
+    }
+  }
   expert_list_prologue(L, list, first + L.E, first, ctl);
   // ---- tokens -> B fragments.  x is an input of the whole block: readable
   //      before this grid waits on the router.

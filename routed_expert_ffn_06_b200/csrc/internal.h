@@ -21,6 +21,8 @@ struct LayerDev {
   const uint16_t* sscales;
   const float* pref;   // selection bonus [E] or nullptr
   float* counts;       // routing counters [E] or nullptr
+  const char* pf[3];   // L2 prefetch ranges (the next layer's router and shared expert)
+  unsigned pfb[3];     // their bytes (multiples of 16; 0 = none)
   long long cbe;   // codes bytes per routed expert
   long long nse;   // scales per routed expert
 };

@@ -47,7 +47,7 @@ moe_status check_device() {
 
 namespace {
 
-moe_status validate_layer(const moe_layer* l) {
+moe_status validate_own(const moe_layer* l) {
   if (!l) return MOE_ERR_INVALID_ARG;
   if (l->group != kGroup) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (l->bits != 2 && l->bits != 3) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -63,6 +63,14 @@ moe_status validate_layer(const moe_layer* l) {
     return MOE_ERR_MISALIGNED;
   if (l->shared_ffn > 0 && (!aligned16(l->shared_codes) || !aligned16(l->shared_scales)))
     return MOE_ERR_MISALIGNED;
+  return MOE_OK;
+}
+
+// The layer, and the next layer named for the L2 prefetch (its own fields only).
+moe_status validate_layer(const moe_layer* l) {
+  const moe_status s = validate_own(l);
+  if (s != MOE_OK) return s;
+  if (l->l2_next && validate_own(l->l2_next) != MOE_OK) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -85,6 +93,19 @@ LayerDev to_dev(const moe_layer* l) {
   L.counts = l->route_counts;
   L.cbe = 3LL * L.F * L.d / kGroup * group_bytes(L.bits);
   L.nse = 3LL * L.F * L.d / kGroup;
+  for (int r = 0; r < 3; ++r) {
+    L.pf[r] = nullptr;
+    L.pfb[r] = 0;
+  }
+  if (const moe_layer* n = l->l2_next) {   // checked by validate_layer
+    const long long sg = 3LL * n->shared_ffn * n->d_model / kGroup;
+    L.pf[0] = reinterpret_cast<const char*>(n->router_w);
+    L.pfb[0] = (unsigned)((long long)n->n_experts * n->d_model * 4);
+    L.pf[1] = reinterpret_cast<const char*>(n->shared_codes);
+    L.pfb[1] = n->shared_codes ? (unsigned)(sg * group_bytes(n->bits)) : 0u;
+    L.pf[2] = reinterpret_cast<const char*>(n->shared_scales);
+    L.pfb[2] = n->shared_scales ? (unsigned)(sg * 2) : 0u;
+  }
   return L;
 }
 

@@ -53,7 +53,7 @@ class moe_layer(ctypes.Structure):
                 ("expert_slot", ctypes.c_void_p), ("codes", ctypes.c_void_p),
                 ("scales", ctypes.c_void_p), ("shared_codes", ctypes.c_void_p),
                 ("shared_scales", ctypes.c_void_p), ("router_pref", ctypes.c_void_p),
-                ("route_counts", ctypes.c_void_p)]
+                ("route_counts", ctypes.c_void_p), ("l2_next", ctypes.c_void_p)]
 
 
 _lib = None
@@ -135,6 +135,22 @@ def make_layer_struct(layer, router_pref=None, route_counts=None) -> moe_layer:
                      _ptr(layer.router_bias), _ptr(layer.expert_slot), _ptr(layer.codes),
                      _ptr(layer.scales), _ptr(layer.shared_codes), _ptr(layer.shared_scales),
                      _ptr(router_pref), _ptr(route_counts))
+
+
+def link_l2_next(structs, cyclic: bool = True) -> None:
+    """Name, in each moe_layer of a sequence, the one run after it (the last
+    names the first when cyclic), so that each decode step prefetches the next
+    layer's router and shared expert into L2.  The structs must outlive the
+    calls (and any graph captured from them)."""
+    n = len(structs)
+    for i, L in enumerate(structs):
+        j = i + 1
+        if j == n:
+            if not cyclic:
+                L.l2_next = None
+                continue
+            j = 0
+        L.l2_next = ctypes.addressof(structs[j])
 
 
 def moe_workspace_bytes(layer: moe_layer, max_tokens: int) -> int:

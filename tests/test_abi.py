@@ -173,3 +173,24 @@ def test_wait_limit_and_withhold_switch_validation(lib):
         assert set_limit(ws, 1 << 20, 60_000_000, None) == 8
         assert set_limit(ws, 1 << 20, 0, None) == 8
         assert set_site(ws, 1 << 20, moe.WITHHOLD_PREFILL_ARRIVE, None) == 8
+
+
+def test_l2_next_layer_is_validated(lib):
+    """A next layer named for the L2 prefetch must pass the layer checks
+    (MOE_ERR_INVALID_ARG otherwise); a valid one lets the call reach the
+    missing device."""
+    x, y, ws = 0x7F0000400000, 0x7F0000500000, 0x7F0000600000
+    L = _layer()
+    bad = _layer(bits=4)
+    L.l2_next = ctypes.addressof(bad)
+    assert lib.moe_block_forward(ctypes.byref(L), x, 4, y, 0, ws, 1 << 30, None) == 1
+    good = _layer(n_experts=32)
+    L.l2_next = ctypes.addressof(good)
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.moe_block_forward(ctypes.byref(L), x, 4, y, 0, ws, 1 << 30, None) == 8
+    structs = [_layer() for _ in range(3)]
+    moe.link_l2_next(structs)
+    assert [s.l2_next for s in structs] == [ctypes.addressof(structs[1]),
+                                            ctypes.addressof(structs[2]),
+                                            ctypes.addressof(structs[0])]

@@ -238,3 +238,30 @@ def test_block_forward_middle_windows(T):
         torch.cuda.synchronize()
         assert torch.equal(y, torch.cat(parts))
     assert gb.error_word() == (0, 0)
+
+
+def test_l2_prefetch_of_the_next_layer_changes_no_result():
+    """Naming the next layer (its router and shared expert prefetched into L2
+    by this layer's expert step) is a hint: outputs equal, byte for byte, the
+    same chain without it, for decode windows and sub-windows."""
+    wl = synth.WORKLOADS["decode_stack"]
+    layers = [synth.make_layer(wl["shape"], seed=0, layer=l, device="cuda", bias=wl["bias"],
+                               slot=wl["slot"]) for l in range(3)]
+    plain = [moe.make_layer_struct(l) for l in layers]
+    linked = [moe.make_layer_struct(l) for l in layers]
+    moe.link_l2_next(linked)
+    flags = moe.F_PRENORM | moe.F_RESIDUAL
+    for T in (1, 4, 12):
+        x = synth.make_tokens(T, 2048, seed=70 + T, device="cuda")
+        outs = []
+        for structs in (plain, linked):
+            ws = moe.alloc_workspace(structs[0], T)
+            h = x
+            for L in structs:
+                y = torch.empty_like(h)
+                moe.moe_block_forward(L, h, T, y, flags, ws)
+                h = y
+            torch.cuda.synchronize()
+            assert moe.moe_workspace_error(ws) == (0, 0)
+            outs.append(h)
+        assert torch.equal(outs[0], outs[1])
