@@ -207,8 +207,8 @@ def measured_traffic(name: str):
 
 # ------------------------------------------------------------------ decode
 DECODE_WINDOWS = (1, 2, 3, 4)
-PREFILL_LAUNCHES = 11       # split router, router GEMM, top-k, prep, hist, scan, scatter,
-                            # gather, GEMM1, GEMM2, combine per 8192-token chunk
+PREFILL_LAUNCHES = 10       # router GEMM, top-k, prep, hist, scan, scatter, gather, GEMM1,
+                            # GEMM2, combine per 8192-token chunk (router split at load)
 WORKLOAD_DECODE = ("decode single layer: d=2048, 512 experts ffn=512 + shared ffn=512, top-10, "
                    "2-bit g32 fp16 scales, Zipf(1.1) popularity, frequency-ordered slots; "
                    "verify windows T=1,2,3,4")
@@ -475,6 +475,10 @@ def measure_prefill(args, rank, world, local, K, W):
     layers = [synth.make_layer(sh, seed=rank * 1000 + i, layer=i, device=dev, bias=wl["bias"],
                                bias_std=wl["bias_std"], slot=wl["slot"]) for i in range(NL)]
     structs = [moe.make_layer_struct(l) for l in layers]
+    # router weights split into bf16 hi/lo once per layer, as at model load
+    splits = [moe.moe_router_split(L) for L in structs]
+    for L, sp in zip(structs, splits):
+        L.router_w_split = sp.data_ptr()
     ws = moe.alloc_workspace(structs[0], T)
     xs = [synth.make_tokens(T, sh.d, seed=rank * 1000 + 3, step=i, device=dev) for i in range(4)]
     y = torch.empty(T, sh.d, dtype=torch.bfloat16, device=dev)
@@ -768,6 +772,9 @@ def bench_mix(args, rank, world, local):
     AE = args.adapt_every
     counts = [torch.zeros(sh.E, dtype=torch.float32, device=dev) if AE else None for _ in layers]
     structs = [moe.make_layer_struct(l, route_counts=c) for l, c in zip(layers, counts)]
+    splits = [moe.moe_router_split(L) for L in structs]   # once per layer, as at model load
+    for L, sp in zip(structs, splits):
+        L.router_w_split = sp.data_ptr()
     if args.l2_next:
         moe.link_l2_next(structs)
     ws = moe.alloc_workspace(structs[0], C)

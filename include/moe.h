@@ -138,7 +138,22 @@ typedef struct moe_layer_s {
    * same way ("Strata illustrated", section on long prompts: the next
    * layer's experts stream in while the current layer computes). */
   const struct moe_layer_s* l2_next;
+  /* dev bf16 bits [2][E][d] or NULL: the router weights split once into
+   * hi = bf16(router_w) followed by lo = bf16(router_w - hi), as written by
+   * moe_router_split().  When given, the tensor-core router of windows above
+   * 8 tokens reads it instead of splitting router_w into the workspace on
+   * every call (same logits, bit for bit).  The caller keeps it in step with
+   * router_w.  16-byte aligned, else MOE_ERR_MISALIGNED. */
+  const uint16_t* router_w_split;
 } moe_layer;
+
+/* Split the layer's fp32 router weights into the bf16 hi and lo parts the
+ * tensor-core router multiplies (out: dev bf16 bits [2][E][d], 16-byte
+ * aligned, caller-owned; enqueued on stream).  Meant for once per layer at
+ * load time: set the result as moe_layer.router_w_split.  The router's
+ * accuracy argument is in the comment of the router for long windows: the
+ * residual of the two terms is below 2^-16 |Wr|. */
+moe_status moe_router_split(const moe_layer* layer, uint16_t* out, void* stream);
 
 /* Bytes of workspace the calls below need for up to max_tokens tokens
  * (0 on invalid arguments).  The decode path (moe_route_topk with T <= 8,

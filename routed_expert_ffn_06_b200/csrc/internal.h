@@ -21,6 +21,7 @@ struct LayerDev {
   const uint16_t* sscales;
   const float* pref;   // selection bonus [E] or nullptr
   float* counts;       // routing counters [E] or nullptr
+  const uint16_t* wsplit;   // router weights split into bf16 hi, lo [2][E][d] or nullptr
   const char* pf[3];   // L2 prefetch ranges (the next layer's router and shared expert)
   unsigned pfb[3];     // their bytes (multiples of 16; 0 = none)
   long long cbe;   // codes bytes per routed expert
@@ -64,7 +65,10 @@ cudaError_t launch_router_large(const LayerDev& L, const uint16_t* x, int T, uin
                                 float* logits, int32_t* ids, float* w, uint16_t* wsplit,
                                 Control* ctl, cudaStream_t st);
 cudaError_t launch_router_tc(const LayerDev& L, const uint16_t* x, int T, float* logits,
-                             uint16_t* hi, uint16_t* lo, Control* ctl, cudaStream_t st);
+                             uint16_t* hi, uint16_t* lo, bool split, Control* ctl,
+                             cudaStream_t st);
+cudaError_t launch_split_router(const float* Wr, int E, int d, uint16_t* hi, uint16_t* lo,
+                                cudaStream_t st);
 bool decode_fits(int d, int E, int Fmax, int bits, int T);
 // Widest window the block forward runs as consecutive decode windows of up
 // to kMaxDecodeT tokens (the measured crossover to the prefill pipeline).

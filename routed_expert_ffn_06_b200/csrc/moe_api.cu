@@ -63,6 +63,7 @@ moe_status validate_own(const moe_layer* l) {
     return MOE_ERR_MISALIGNED;
   if (l->shared_ffn > 0 && (!aligned16(l->shared_codes) || !aligned16(l->shared_scales)))
     return MOE_ERR_MISALIGNED;
+  if (l->router_w_split && !aligned16(l->router_w_split)) return MOE_ERR_MISALIGNED;
   return MOE_OK;
 }
 
@@ -91,6 +92,7 @@ LayerDev to_dev(const moe_layer* l) {
   L.sscales = l->shared_scales;
   L.pref = l->router_pref;
   L.counts = l->route_counts;
+  L.wsplit = l->router_w_split;
   L.cbe = 3LL * L.F * L.d / kGroup * group_bytes(L.bits);
   L.nse = 3LL * L.F * L.d / kGroup;
   for (int r = 0; r < 3; ++r) {
@@ -288,6 +290,17 @@ moe_status moe_workspace_error(void* ws, size_t ws_bytes, uint32_t* code_out, vo
   if (code & kErrTimeout) return MOE_ERR_TIMEOUT;
   if (code) return MOE_ERR_DEVICE_CHECK;
   return MOE_OK;
+}
+
+moe_status moe_router_split(const moe_layer* layer, uint16_t* out, void* stream) {
+  moe_status s = validate_layer(layer);
+  if (s != MOE_OK) return s;
+  if (!out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out)) return MOE_ERR_MISALIGNED;
+  if ((s = check_device()) != MOE_OK) return s;
+  const size_t n = (size_t)layer->n_experts * layer->d_model;
+  return from_cuda(launch_split_router(layer->router_w, layer->n_experts, layer->d_model, out,
+                                       out + n, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_workspace_set_wait_limit(void* ws, size_t ws_bytes, uint32_t limit_us,

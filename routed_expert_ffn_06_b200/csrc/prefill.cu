@@ -1025,39 +1025,51 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const PfArgs a,
 // row of t] (+ x[t])), the routed terms in selection order and the shared
 // expert last, in fp32; every term already carries its routing weight.  The
 // fixed order makes the result independent of scheduling.  One warp per
-// token, 8 elements (16 bytes of fp16) per lane and step.
+// token, 8 elements (16 bytes of fp16) per lane and step; the terms' loads
+// are issued four at a time (their positions staged in shared memory), so
+// their latencies overlap while the sum keeps its order.
 __global__ void __launch_bounds__(256) prefill_combine_kernel(
     const __half* __restrict__ ybuf, const int* __restrict__ invpos, const int* __restrict__ offsets,
     const uint16_t* __restrict__ x, int T, int d, int k, int E, int has_shared, uint32_t flags,
     uint16_t* __restrict__ y) {
+  __shared__ int spos[8][17];   // per warp: the token's k routed positions, then the shared one
   pdl_wait();
   pdl_launch_dependents();
   const int per = d / 8;
   const int sh0 = offsets[E];
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int nw = gridDim.x * (blockDim.x >> 5);
-  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nw) {
-    const int mypos = lane < k ? invpos[(size_t)t * k + lane] : -1;
+  const int nt = k + 1;
+  for (int t = blockIdx.x * (blockDim.x >> 5) + wib; t < T; t += nw) {
+    __syncwarp();
+    if (lane < k) spos[wib][lane] = invpos[(size_t)t * k + lane];
+    if (lane == 0) spos[wib][k] = has_shared ? sh0 + t : -1;
+    __syncwarp();
     for (int c = lane; c < per; c += 32) {
       float v[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = 0.f;
-      for (int j = 0; j <= k; ++j) {
-        int pos;
-        if (j < k) {
-          pos = __shfl_sync(0xffffffffu, mypos, j);
-        } else {
-          if (!has_shared) break;
-          pos = sh0 + t;
-        }
-        if (pos < 0) continue;
-        const uint4 u = reinterpret_cast<const uint4*>(ybuf + (size_t)pos * d)[c];
-        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+      // the terms in a fixed order (selection order, shared expert last; -1:
+      // no term), loaded four at a time so that their latencies overlap
+      for (int j0 = 0; j0 < nt; j0 += 4) {
+        uint4 u[4];
+        int pq[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(u32_as_h2(w4[e]));
-          v[2 * e] += f.x;
-          v[2 * e + 1] += f.y;
+        for (int q = 0; q < 4; ++q) {
+          pq[q] = j0 + q < nt ? spos[wib][j0 + q] : -1;
+          u[q] = pq[q] >= 0 ? reinterpret_cast<const uint4*>(ybuf + (size_t)pq[q] * d)[c]
+                            : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (pq[q] < 0) continue;
+          const uint32_t w4[4] = {u[q].x, u[q].y, u[q].z, u[q].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(u32_as_h2(w4[e]));
+            v[2 * e] += f.x;
+            v[2 * e + 1] += f.y;
+          }
         }
       }
       const size_t i = (size_t)t * per + c;

@@ -170,7 +170,9 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerDev L, const float* __re
 cudaError_t launch_router_large(const LayerDev& L, const uint16_t* x, int T, uint32_t flags,
                                 float* logits, int32_t* ids, float* w, uint16_t* wsplit,
                                 Control* ctl, cudaStream_t st) {
-  cudaError_t e = launch_router_tc(L, x, T, logits, wsplit, wsplit + (size_t)L.E * L.d, ctl, st);
+  // the caller's split router weights when given, else split into the workspace
+  uint16_t* hi = L.wsplit ? const_cast<uint16_t*>(L.wsplit) : wsplit;
+  cudaError_t e = launch_router_tc(L, x, T, logits, hi, hi + (size_t)L.E * L.d, !L.wsplit, ctl, st);
   if (e != cudaSuccess) return e;
   return launch_pdl(topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, L,
                     static_cast<const float*>(logits), T, ids, w, flags, ctl);

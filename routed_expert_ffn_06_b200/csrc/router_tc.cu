@@ -180,14 +180,25 @@ __global__ void __launch_bounds__(RT_THREADS, 1) router_tc_kernel(const float* _
 size_t router_tc_smem() { return (size_t)RT_STAGES * RT_STAGE + 2 * RT_STAGES * 8 + 8 + 16 + 1024; }
 
 // hi/lo: workspace [E][d] bf16 each.  x: bf16 [T][d] (16-byte aligned).
-cudaError_t launch_router_tc(const LayerDev& L, const uint16_t* x, int T, float* logits,
-                             uint16_t* hi, uint16_t* lo, Control* ctl, cudaStream_t st) {
-  const long long n4 = (long long)L.E * L.d / 4;
+cudaError_t launch_split_router(const float* Wr, int E, int d, uint16_t* hi, uint16_t* lo,
+                                cudaStream_t st) {
+  const long long n4 = (long long)E * d / 4;
   int g = (int)((n4 + 255) / 256);
   if (g > 2 * sm_count()) g = 2 * sm_count();
-  cudaError_t e = launch_pdl(split_router_kernel, dim3(g), dim3(256), 0, st, L.Wr, n4,
-                             reinterpret_cast<uint2*>(hi), reinterpret_cast<uint2*>(lo));
-  if (e != cudaSuccess) return e;
+  return launch_pdl(split_router_kernel, dim3(g), dim3(256), 0, st, Wr, n4,
+                    reinterpret_cast<uint2*>(hi), reinterpret_cast<uint2*>(lo));
+}
+
+// hi/lo: [E][d] bf16 each; split = true writes them from Wr first (otherwise
+// they hold the split already).
+cudaError_t launch_router_tc(const LayerDev& L, const uint16_t* x, int T, float* logits,
+                             uint16_t* hi, uint16_t* lo, bool split, Control* ctl,
+                             cudaStream_t st) {
+  cudaError_t e = cudaSuccess;
+  if (split) {
+    e = launch_split_router(L.Wr, L.E, L.d, hi, lo, st);
+    if (e != cudaSuccess) return e;
+  }
   RtMaps mp;
   if (!make_map_b16(&mp.hi, hi, (uint64_t)L.d, (uint64_t)L.E) ||
       !make_map_b16(&mp.lo, lo, (uint64_t)L.d, (uint64_t)L.E) ||

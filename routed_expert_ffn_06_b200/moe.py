@@ -33,7 +33,8 @@ F_DEBUG = 8
 WITHHOLD_PREFILL_ARRIVE = 1
 
 EXPORTS = ["moe_workspace_bytes", "moe_workspace_init", "moe_workspace_error",
-           "moe_workspace_set_wait_limit", "moe_workspace_set_debug_withhold", "moe_route_topk",
+           "moe_workspace_set_wait_limit", "moe_workspace_set_debug_withhold", "moe_router_split",
+           "moe_route_topk",
            "moe_expert_ffn_decode", "moe_expert_ffn_prefill", "moe_block_forward",
            "moe_block_forward_noalloc", "moe_adapt_workspace_bytes", "moe_adapt_layout",
            "moe_status_string", "moe_build_info", "moe_pack_host"]
@@ -53,7 +54,8 @@ class moe_layer(ctypes.Structure):
                 ("expert_slot", ctypes.c_void_p), ("codes", ctypes.c_void_p),
                 ("scales", ctypes.c_void_p), ("shared_codes", ctypes.c_void_p),
                 ("shared_scales", ctypes.c_void_p), ("router_pref", ctypes.c_void_p),
-                ("route_counts", ctypes.c_void_p), ("l2_next", ctypes.c_void_p)]
+                ("route_counts", ctypes.c_void_p), ("l2_next", ctypes.c_void_p),
+                ("router_w_split", ctypes.c_void_p)]
 
 
 _lib = None
@@ -77,6 +79,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.moe_workspace_init.argtypes = [vp, sz, vp]
     L.moe_workspace_error.restype = st
     L.moe_workspace_error.argtypes = [vp, sz, ctypes.POINTER(u32), vp]
+    L.moe_router_split.restype = st
+    L.moe_router_split.argtypes = [P, vp, vp]
     L.moe_workspace_set_wait_limit.restype = st
     L.moe_workspace_set_wait_limit.argtypes = [vp, sz, u32, vp]
     L.moe_workspace_set_debug_withhold.restype = st
@@ -135,6 +139,16 @@ def make_layer_struct(layer, router_pref=None, route_counts=None) -> moe_layer:
                      _ptr(layer.router_bias), _ptr(layer.expert_slot), _ptr(layer.codes),
                      _ptr(layer.scales), _ptr(layer.shared_codes), _ptr(layer.shared_scales),
                      _ptr(router_pref), _ptr(route_counts))
+
+
+def moe_router_split(layer: moe_layer, stream=None) -> torch.Tensor:
+    """The layer's router weights split into bf16 hi and lo parts ([2][E][d],
+    bf16 bits as int16) on the current device; set it as
+    layer.router_w_split (keep the tensor alive while the struct is used)."""
+    out = torch.empty(2, layer.n_experts, layer.d_model, dtype=torch.int16, device="cuda")
+    _check(load().moe_router_split(ctypes.byref(layer), _ptr(out), _stream(stream)),
+           "moe_router_split")
+    return out
 
 
 def link_l2_next(structs, cyclic: bool = True) -> None:

@@ -194,3 +194,19 @@ def test_l2_next_layer_is_validated(lib):
     assert [s.l2_next for s in structs] == [ctypes.addressof(structs[1]),
                                             ctypes.addressof(structs[2]),
                                             ctypes.addressof(structs[0])]
+
+
+def test_router_split_validation(lib):
+    """moe_router_split checks the layer and its output pointer on the host;
+    a misaligned pre-split router in the layer is rejected by every call."""
+    L = _layer()
+    out = 0x7F0000900000
+    assert lib.moe_router_split(ctypes.byref(L), None, None) == 1
+    assert lib.moe_router_split(ctypes.byref(L), out + 2, None) == 4
+    assert lib.moe_router_split(ctypes.byref(_layer(bits=4)), out, None) == 2
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.moe_router_split(ctypes.byref(L), out, None) == 8
+    L.router_w_split = out + 8
+    x, y, ws = 0x7F0000400000, 0x7F0000500000, 0x7F0000600000
+    assert lib.moe_block_forward(ctypes.byref(L), x, 64, y, 0, ws, 1 << 30, None) == 4

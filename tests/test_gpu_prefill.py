@@ -209,6 +209,32 @@ def test_router_large_T_tensor_core(T, d, E):
     assert gb.error_word() == (0, 0)
 
 
+@pytest.mark.parametrize("T,d,E", [(9, 64, 16), (300, 96, 40), (1000, 2048, 512)])
+def test_router_presplit_weights_give_the_same_routing(T, d, E):
+    """Router weights split once by moe_router_split and handed over as
+    router_w_split: the same logits, ids and weights, bit for bit, as the
+    split the router makes in the workspace on every call; and the split
+    itself is hi = bf16(Wr), lo = bf16(Wr - hi) (torch's round to nearest
+    even)."""
+    sh = synth.MoEShape(d=d, E=E, F=64, Fs=0, k=min(10, E // 2), bits=2)
+    layer = synth.make_layer(sh, seed=T + 7, device="cuda", bias="normal")
+    x = synth.make_tokens(T, d, seed=T + 8, device="cuda")
+    gb = GpuBlock(layer, T)
+    ref = gb.route(x)
+    split = moe.moe_router_split(gb.L)
+    gb.L.router_w_split = split.data_ptr()
+    got = gb.route(x)
+    torch.cuda.synchronize()
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b)
+    wr = layer.router_w.float()
+    hi = wr.to(torch.bfloat16)
+    lo = (wr - hi.float()).to(torch.bfloat16)
+    assert torch.equal(split[0], hi.view(torch.int16))
+    assert torch.equal(split[1], lo.view(torch.int16))
+    assert gb.error_word() == (0, 0)
+
+
 def test_prefill_hot_experts_split_into_many_chunks():
     """Every token routes to the same k experts (router bias far above the
     token logits), so k buckets hold all T tokens, several 128-token chunks
