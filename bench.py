@@ -57,9 +57,9 @@ def parse():
     p.add_argument("--adapt-decay", type=float, default=0.5)
     p.add_argument("--rounds", type=int, default=2048,
                    help="rounds of the T=1..4 windows in one decode step (smaller for profiling)")
-    p.add_argument("--no-l2-next", dest="l2_next", action="store_false",
-                   help="do not let each decode step prefetch the next layer's router and shared "
-                        "expert into L2")
+    p.add_argument("--l2-next", action="store_true",
+                   help="each decode step prefetches the next layer's router and shared expert "
+                        "into L2 (its bytes then count in that step's DRAM traffic)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-prefill", action="store_true",
                    help="decode workload only (no prefill object in the line)")
@@ -429,7 +429,7 @@ def bench_decode(args, rank, world, local):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "traffic": measured_traffic("decode_expert_step"), "peak_src": peaks["src"],
-                     "kernel": "expert step (decode_expert_kernel + decode_combine_kernel per "
+                     "kernel": "expert step (decode_gu_kernel + decode_dn_kernel per "
                                "moe_expert_ffn_decode call)",
                      "bytes_per_launch": round(exp_bytes / n_exp),
                      "us_per_launch_by_T": per_T,
