@@ -210,3 +210,13 @@ def test_router_split_validation(lib):
     L.router_w_split = out + 8
     x, y, ws = 0x7F0000400000, 0x7F0000500000, 0x7F0000600000
     assert lib.moe_block_forward(ctypes.byref(L), x, 64, y, 0, ws, 1 << 30, None) == 4
+
+
+def test_middle_windows_of_a_wide_layer_take_the_prefill_step(lib):
+    """Windows of 9..32 tokens use the decode kernels only for layers within
+    their width: with ffn 4096 at d 256 a 16-token window takes the prefill
+    step and needs the whole workspace (one byte short is too small)."""
+    x, y = 0x7F0000400000, 0x7F0000500000
+    L = _layer(d_model=256, n_experts=20, ffn=4096, shared_ffn=4096, top_k=16)
+    full = lib.moe_workspace_bytes(ctypes.byref(L), 16)
+    assert lib.moe_block_forward(ctypes.byref(L), x, 16, y, 0, 0x7F0000600000, full - 1, None) == 3

@@ -265,3 +265,28 @@ def test_l2_prefetch_of_the_next_layer_changes_no_result():
             assert moe.moe_workspace_error(ws) == (0, 0)
             outs.append(h)
         assert torch.equal(outs[0], outs[1])
+
+
+@pytest.mark.parametrize("T", [12, 32])
+def test_block_forward_middle_windows_prenorm_residual(T):
+    """The middle windows with pre-norm and residual (the stack's flags) on
+    the 3-bit layer: byte-equal to explicit decode calls on the 8-token pieces,
+    and within tolerance of the oracle."""
+    wl = synth.WORKLOADS["decode_stack"]
+    layer = synth.make_layer(wl["shape"], seed=0, layer=3, device="cuda", bias=wl["bias"],
+                             slot=wl["slot"])
+    x = (synth.make_tokens(T, 2048, seed=90 + T, device="cuda").float() * 3).to(torch.bfloat16)
+    flags = moe.F_PRENORM | moe.F_RESIDUAL
+    gb = GpuBlock(layer, T)
+    y = gb.block(x, flags)
+    parts, routed = [], []
+    for t0 in range(0, T, 8):   # the router of each 8-token piece, as the block runs it
+        xs = x[t0:t0 + 8].clone()
+        r = gb.route(xs, flags)
+        routed.append(r)
+        parts.append(gb.decode(xs, r[1], r[2], flags))
+    torch.cuda.synchronize()
+    assert torch.equal(y, torch.cat(parts))
+    logits, ids, w = (torch.cat([r[i] for r in routed]) for i in range(3))
+    oracle_check(layer, x, logits, ids, w, y, flags=flags)
+    assert gb.error_word() == (0, 0)
