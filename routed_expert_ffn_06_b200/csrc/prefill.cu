@@ -201,12 +201,19 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(int* __restrict__ blo
   pdl_wait();
   pdl_launch_dependents();
   const int tid = threadIdx.x;
+  // per expert, the exclusive running sum over token blocks; the block
+  // counts are loaded 16 at a time so that their latencies overlap
   for (int e = tid; e < E; e += blockDim.x) {
     int run = 0;
-    for (int b = 0; b < nblk; ++b) {
-      const int c = blockcnt[(size_t)b * E + e];
-      blockcnt[(size_t)b * E + e] = run;
-      run += c;
+    for (int b0 = 0; b0 < nblk; b0 += 16) {
+      int c[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) c[j] = b0 + j < nblk ? blockcnt[(size_t)(b0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (b0 + j < nblk) blockcnt[(size_t)(b0 + j) * E + e] = run;
+        run += c[j];
+      }
     }
     cnt[e] = run;
   }
