@@ -163,7 +163,8 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerDev L, const float* __re
   pdl_launch_dependents();
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
-  warp_topk(logits + (size_t)t * L.E, L.pref, L.counts, L.E, L.k, ids + (size_t)t * L.k, w + (size_t)t * L.k, ctl,
+  // the lean rescan: fewer registers, more warps of this batch kernel resident
+  warp_topk<true>(logits + (size_t)t * L.E, L.pref, L.counts, L.E, L.k, ids + (size_t)t * L.k, w + (size_t)t * L.k, ctl,
             flags & MOE_F_DEBUG);
 }
 

@@ -20,8 +20,11 @@ constexpr float kRmsEps = 1e-6f;
 // its own logits (ties: lowest index, as the lane scans upward); a round takes
 // the warp maximum of the keys and the lowest index holding it (two redux
 // instructions), and only the winning lane rescans.  NPER >= E / 32 logits per
-// lane.
-template <int NPER, bool PREF>
+// lane.  LEAN picks how a lane rescans: a running comparison (few registers,
+// for the batch top-k kernel whose occupancy they limit) or a tree over
+// packed (key, ~index) pairs (a shorter dependency chain per round, for the
+// latency of one small window).  Both choose the same entry.
+template <int NPER, bool PREF, bool LEAN = false>
 __device__ void warp_topk_n(const float* __restrict__ row, const float* __restrict__ pref,
                             float* __restrict__ counts, int E, int k, int32_t* __restrict__ ids,
                             float* __restrict__ w, Control* ctl, bool debug) {
@@ -46,28 +49,42 @@ __device__ void warp_topk_n(const float* __restrict__ row, const float* __restri
   }
   if (debug && bad) record_error(ctl, kErrNonFinite, 0x100);
   uint32_t taken = 0;
-  // lane-local best by a depth-5 tree over (key << 32 | ~index): larger key
-  // wins, equal keys go to the lower index; 0 marks invalid or taken entries
+  // lane-local best: a scan in ascending expert index in which only a
+  // strictly larger key replaces the best, so equal keys stay with the lower
+  // index (a NaN, key 0, wins only where nothing else is left); bi =
+  // 0xFFFFFFFF when every entry of the lane is taken or outside E
   uint32_t bk = 0u, bi = 0xFFFFFFFFu;
   auto rescan = [&]() {
-    unsigned long long c[NPER];
+    if constexpr (LEAN) {
+      uint32_t k0 = 0u, i0 = 0xFFFFFFFFu;
 #pragma unroll
-    for (int i = 0; i < NPER; ++i) {
-      const uint32_t e = (uint32_t)(lane + 32 * i);
-      const bool ok = ((int)e < E) && !((taken >> i) & 1u);
-      c[i] = ok ? ((unsigned long long)key[i] << 32) | (unsigned long long)(~e) : 0ull;
-    }
-#pragma unroll
-    for (int half = NPER / 2; half >= 1; half >>= 1) {
-#pragma unroll
-      for (int i = 0; i < half; ++i) c[i] = c[i + half] > c[i] ? c[i + half] : c[i];
-    }
-    if (c[0] == 0ull) {
-      bk = 0u;
-      bi = 0xFFFFFFFFu;
+      for (int i = 0; i < NPER; ++i) {
+        const uint32_t e = (uint32_t)(lane + 32 * i);
+        const bool ok = ((int)e < E) && !((taken >> i) & 1u);
+        if (ok && (i0 == 0xFFFFFFFFu || key[i] > k0)) {
+          k0 = key[i];
+          i0 = e;
+        }
+      }
+      bk = k0;
+      bi = i0;
     } else {
-      bk = (uint32_t)(c[0] >> 32);
-      bi = ~(uint32_t)(c[0] & 0xFFFFFFFFull);
+      // (key << 32 | ~index): the larger key wins, equal keys go to the lower
+      // index; 0 marks an entry that is taken or outside E
+      unsigned long long c[NPER];
+#pragma unroll
+      for (int i = 0; i < NPER; ++i) {
+        const uint32_t e = (uint32_t)(lane + 32 * i);
+        const bool ok = ((int)e < E) && !((taken >> i) & 1u);
+        c[i] = ok ? ((unsigned long long)key[i] << 32) | (unsigned long long)(~e) : 0ull;
+      }
+#pragma unroll
+      for (int half = NPER / 2; half >= 1; half >>= 1) {
+#pragma unroll
+        for (int i = 0; i < half; ++i) c[i] = c[i + half] > c[i] ? c[i + half] : c[i];
+      }
+      bk = c[0] ? (uint32_t)(c[0] >> 32) : 0u;
+      bi = c[0] ? ~(uint32_t)(c[0] & 0xFFFFFFFFull) : 0xFFFFFFFFu;
     }
   };
   rescan();
@@ -112,33 +129,34 @@ __device__ void warp_topk_n(const float* __restrict__ row, const float* __restri
 
 // The variants with a selection bonus are kept out of line: their extra
 // register arrays then leave the plain path's allocation alone.
-template <int NPER>
+template <int NPER, bool LEAN>
 __device__ __noinline__ void warp_topk_pref(const float* __restrict__ row,
                                             const float* __restrict__ pref,
                                             float* __restrict__ counts, int E, int k,
                                             int32_t* __restrict__ ids, float* __restrict__ w,
                                             Control* ctl, bool debug) {
-  warp_topk_n<NPER, true>(row, pref, counts, E, k, ids, w, ctl, debug);
+  warp_topk_n<NPER, true, LEAN>(row, pref, counts, E, k, ids, w, ctl, debug);
 }
 
+template <bool LEAN = false>
 __device__ __forceinline__ void warp_topk(const float* __restrict__ row, const float* __restrict__ pref,
                                           float* __restrict__ counts, int E, int k,
                                           int32_t* __restrict__ ids, float* __restrict__ w,
                                           Control* ctl, bool debug) {
   if (pref) {
     if (E <= 128)
-      warp_topk_pref<4>(row, pref, counts, E, k, ids, w, ctl, debug);
+      warp_topk_pref<4, LEAN>(row, pref, counts, E, k, ids, w, ctl, debug);
     else if (E <= 512)
-      warp_topk_pref<16>(row, pref, counts, E, k, ids, w, ctl, debug);
+      warp_topk_pref<16, LEAN>(row, pref, counts, E, k, ids, w, ctl, debug);
     else
-      warp_topk_pref<32>(row, pref, counts, E, k, ids, w, ctl, debug);
+      warp_topk_pref<32, LEAN>(row, pref, counts, E, k, ids, w, ctl, debug);
   } else {
     if (E <= 128)
-      warp_topk_n<4, false>(row, pref, counts, E, k, ids, w, ctl, debug);
+      warp_topk_n<4, false, LEAN>(row, pref, counts, E, k, ids, w, ctl, debug);
     else if (E <= 512)
-      warp_topk_n<16, false>(row, pref, counts, E, k, ids, w, ctl, debug);
+      warp_topk_n<16, false, LEAN>(row, pref, counts, E, k, ids, w, ctl, debug);
     else
-      warp_topk_n<32, false>(row, pref, counts, E, k, ids, w, ctl, debug);
+      warp_topk_n<32, false, LEAN>(row, pref, counts, E, k, ids, w, ctl, debug);
   }
 }
 
