@@ -1,6 +1,7 @@
 // select.cuh -- per-token top-k selection with softmax renormalisation, and
 // staging of a token window (optional RMSNorm) into shared memory; used by the
-// small-T router and the fused decode kernel.
+// small-window router (selection in its last CTA) and the batch top-k kernel
+// of long windows.
 //
 // Selection: the router keeps the top_k of the expert scores ("Strata
 // open-source runtime", section "the model itself": 10 of 512 per layer);
