@@ -220,3 +220,28 @@ def test_middle_windows_of_a_wide_layer_take_the_prefill_step(lib):
     L = _layer(d_model=256, n_experts=20, ffn=4096, shared_ffn=4096, top_k=16)
     full = lib.moe_workspace_bytes(ctypes.byref(L), 16)
     assert lib.moe_block_forward(ctypes.byref(L), x, 16, y, 0, 0x7F0000600000, full - 1, None) == 3
+
+
+def test_header_compiles_as_c99_and_ctypes_mirrors_moe_layer(tmp_path):
+    """include/moe.h is a C header: it compiles as strict C99, and the ctypes
+    mirror of moe_layer in the binding has the C struct's size and field
+    offsets (measured by a program compiled against the header)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    fields = [f for f, _ in moe.moe_layer._fields_]
+    src = ["#include <stddef.h>", "#include <stdint.h>", "#include <stdio.h>", '#include "moe.h"',
+           "int main(void) {", '  printf("%zu\\n", sizeof(moe_layer));']
+    src += [f'  printf("%zu\\n", offsetof(moe_layer, {f}));' for f in fields]
+    src += ["  return 0;", "}"]
+    c = tmp_path / "layout.c"
+    c.write_text("\n".join(src) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe)], check=True)
+    out = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True,
+                                          text=True).stdout.split()]
+    assert out[0] == ctypes.sizeof(moe.moe_layer)
+    assert out[1:] == [getattr(moe.moe_layer, f).offset for f in fields]
